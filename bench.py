@@ -1,0 +1,356 @@
+#!/usr/bin/env python3
+"""Benchmark: causal CP-attention forward TFLOP/s on B200 (one JSON line on rank 0).
+
+Default workload: Llama-3-8B-shaped GQA ring attention at L = 212992 (208K), 32 query heads,
+8 KV heads, d = 128, N_cp = 16 virtual ranks on one GPU, bf16 inputs i.i.d. N(0,1) from a
+fixed seed.  One step = one cp_attn_fwd call (the whole hot path: every ring step of every
+virtual rank, the online-softmax merges and the bf16 output cast) on inputs already resident
+in HBM.  Inputs (Q 1.6 GiB, K/V 0.4 GiB each) are larger than the 126 MB L2, so no flush is
+needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload c3]
+
+Multi-GPU: the benchmark spec keeps every virtual rank of the problem on one GPU, so N > 1 runs
+N independent replicas (one per GPU, weak scaling); value = total FLOPs / max-over-ranks time.
+--impl reference times the fp64 CPU oracle on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal CP-attention fwd TFLOP/s (1 B200) and % of dense BF16 peak, L=208K"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="c3")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU work of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sequence_long_context_ring_b200", "csrc")
+    for fn in ("fwd_kernel.cuh", "sm100.cuh"):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(workload_name: str):
+    """DRAM bytes per launch of the forward kernel from the committed ncu summary, or None
+    when there is none or the kernel source changed since it was captured."""
+    p = os.path.join(ROOT, "profiles", "ring_fwd_kernel_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    per = d.get("per_launch_bytes", {}).get(workload_name)
+    return float(per) if per is not None else None
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle sampling during the timed region."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+def cpu_oracle_sample(w, target_seconds: float):
+    """Time the fp64 oracle on a bounded sample of the workload: whole query rows of every head
+    (each row exact by the definition), growing the row count until ~target_seconds of work.
+    Returns (TFLOP/s, seconds, rows, cores, description)."""
+    import oracle
+    from sequence_long_context_ring_b200 import synth
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    G = w.Hq // w.Hkv
+    rng = np.random.default_rng(12345)
+    # one KV head and its G query heads, drawn from the same seeded generator layout
+    kv_head = 0
+    k = synth.normal_bf16(w.cfg_id, synth.TENSOR_ID["k"], w.kv_shape(), w.input_scale)
+    v = synth.normal_bf16(w.cfg_id, synth.TENSOR_ID["v"], w.kv_shape(), w.input_scale)
+    q = synth.normal_bf16(w.cfg_id, synth.TENSOR_ID["q"], w.q_shape(), w.input_scale)
+    if w.seq_major:
+        kh = synth.bf16_bits_to_f64(k[0, :, kv_head])
+        vh = synth.bf16_bits_to_f64(v[0, :, kv_head])
+        qsel = lambda h, rows: synth.bf16_bits_to_f64(q[0, rows, h])  # noqa: E731
+    else:
+        kh = synth.bf16_bits_to_f64(k[0, kv_head])
+        vh = synth.bf16_bits_to_f64(v[0, kv_head])
+        qsel = lambda h, rows: synth.bf16_bits_to_f64(q[0, h, rows])  # noqa: E731
+    del q, k, v
+    n_rows, flops, elapsed, total_rows = 8, 0.0, 0.0, 0
+    while elapsed < target_seconds:
+        rows = np.sort(rng.integers(0, w.L, n_rows))
+        t0 = time.perf_counter()
+        for h in range(kv_head * G, kv_head * G + G):
+            oracle.attention_rows(qsel(h, rows), kh, vh, rows, causal=True)
+        dt = time.perf_counter() - t0
+        elapsed += dt
+        flops += G * float(np.sum(4.0 * w.d * (rows + 1)))
+        total_rows += G * n_rows
+        if dt < target_seconds / 4:
+            n_rows *= 2
+    desc = (f"{total_rows} sampled query rows (random positions, full causal key prefix each) of "
+            f"{G} query heads sharing KV head 0 of {w.name}; fp64 numpy oracle")
+    return flops / elapsed / 1e12, elapsed, total_rows, cores, desc
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    t_steps = []
+    value = None
+    desc = cores = None
+    for i in range(args.warmup + args.steps):
+        tflops, sec, rows, cores, desc = cpu_oracle_sample(w, max(2.0, min(args.cpu_seconds, 60.0) / 4))
+        if i >= args.warmup:
+            t_steps.append(sec)
+            value = tflops if value is None else value + tflops
+    value = value / max(1, args.steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(t_steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded bf16 N(0,1), rows sampled)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d,
+                   "n_cp": w.n_cp, "mode": w.mode, "causal": w.causal},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from sequence_long_context_ring_b200 import synth
+    from sequence_long_context_ring_b200.binding import Plan
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # inputs: identical seeded data on every replica
+    def up(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    qb = synth.normal_bf16(w.cfg_id, synth.TENSOR_ID["q"], w.q_shape(), w.input_scale)
+    kb = synth.normal_bf16(w.cfg_id, synth.TENSOR_ID["k"], w.kv_shape(), w.input_scale)
+    vb = synth.normal_bf16(w.cfg_id, synth.TENSOR_ID["v"], w.kv_shape(), w.input_scale)
+    q, k, v = up(qb), up(kb), up(vb)
+    plan = Plan(w.B, w.Hq, w.Hkv, w.L, w.d, n_cp=w.n_cp, n_hp=w.n_hp, mode=w.mode, causal=w.causal)
+    o = torch.empty(w.q_shape(), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+    ws = plan.workspace(False, dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = plan.flops(False)
+
+    for _ in range(args.warmup):
+        plan.fwd(q, k, v, o, lse, ws, stream)
+    torch.cuda.synchronize(dev)
+    st, word = plan.device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} (word {word:#x}) after warm-up")
+
+    # ---- device-timed region: K steps, inputs resident in HBM ----
+    clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev[0].record(stream)
+    for i in range(args.steps):
+        plan.fwd(q, k, v, o, lse, ws, stream)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier()
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    st, word = plan.device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} (word {word:#x}) in the timed region")
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    value = world * flops * args.steps / (max_ms / 1e3) / 1e12
+
+    # ---- end-to-end through the public API with host buffers ----
+    qh, kh, vh = (torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).pin_memory()
+                  for b in (qb, kb, vb))
+    oh = torch.empty(w.q_shape(), dtype=torch.bfloat16).pin_memory()
+    lh = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        plan.fwd(qd, kd, vd, o, lse, ws, stream)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * flops * args.e2e_steps / (float(te.item()) / 1e3) / 1e12
+    h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    # ---- roofline of the dominant kernel (ring mode: one fused launch per step) ----
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    launch_ms = statistics.mean(per_step) if w.mode == "ring" else None
+    roof = None
+    if launch_ms:
+        achieved = flops / (launch_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": traffic_from_profile(w.name),
+                "kernel": "ring_fwd_kernel<128>",
+                "peak_source": f"{peak_src} bf16_tflops_sustained (seconds-long back-to-back launches)"}
+    launches = args.steps * (1 if w.mode == "ring" else 5)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, sec, rows, cores, desc = cpu_oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc, "seconds": sec}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded bf16 N(0,1), Llama-3-8B-shaped)",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d,
+                       "n_cp": w.n_cp, "n_hp": w.n_hp, "mode": w.mode, "causal": w.causal,
+                       "parallelism": f"{world} independent replica(s), all virtual ranks on each GPU",
+                       "l2": "inputs larger than L2 (Q 1.6 GiB), no flush"},
+            "pct_of_peak": 100.0 * (flops / (max_ms / args.steps / 1e3) / 1e12) / peak,
+            "per_step_ms": per_step,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": args.e2e_steps},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    from sequence_long_context_ring_b200.configs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,235 @@
+"""ctypes binding of libcpattn.so (argument marshalling only: every step runs in the CUDA kernels).
+
+Names follow the C ABI in include/cp_attn.h.  torch tensors are passed as strided views
+(data pointer, shape, strides in elements); streams default to torch's current stream.
+There is no fallback: if the library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcpattn.so")
+_lib = None
+
+CP_OK, CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED, CP_ERR_ALIGNMENT = 0, -1, -2, -3
+CP_ERR_WORKSPACE, CP_ERR_CUDA, CP_ERR_TIMEOUT = -4, -5, -6
+CP_BF16, CP_FP32 = 0, 1
+MODES = {"ring": 0, "ulysses": 1, "2d": 2}
+SPLITS = {"contiguous": 0, "zigzag": 1}
+
+
+class CpError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib().cp_status_string(status).decode()} ({status})")
+
+
+class CpTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int), ("ndim", ctypes.c_int),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class CpConfig(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("L", ctypes.c_int),
+                ("d", ctypes.c_int), ("n_cp", ctypes.c_int), ("n_hp", ctypes.c_int), ("causal", ctypes.c_int),
+                ("mode", ctypes.c_int), ("split", ctypes.c_int), ("softmax_scale", ctypes.c_float),
+                ("wait_limit_ns", ctypes.c_uint64), ("debug_fault", ctypes.c_int)]
+
+
+EXPORTS = [
+    "cp_attn_plan", "cp_attn_plan_destroy", "cp_attn_workspace_size", "cp_attn_fwd", "cp_attn_bwd",
+    "cp_layout_seq2head", "cp_layout_head2seq", "cp_ring_step", "cp_lse_merge", "cp_device_status",
+    "cp_status_string", "cp_plan_step_chunk", "cp_plan_flops", "cp_plan_num_work_items", "cp_version",
+]
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcpattn.so (built in-tree by ``sequence_long_context_ring_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libcpattn.so not found at {_LIB_PATH}; run sequence_long_context_ring_b200/build.py")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, T = ctypes.c_void_p, ctypes.POINTER(CpTensor)
+        sig = {
+            "cp_attn_plan": ([ctypes.POINTER(CpConfig), ctypes.POINTER(ctypes.c_void_p)], ctypes.c_int),
+            "cp_attn_plan_destroy": ([P], None),
+            "cp_attn_workspace_size": ([P, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+            "cp_attn_fwd": ([P, T, T, T, T, T, P, ctypes.c_size_t, P], ctypes.c_int),
+            "cp_attn_bwd": ([P, T, T, T, T, T, T, T, T, T, P, ctypes.c_size_t, P], ctypes.c_int),
+            "cp_layout_seq2head": ([ctypes.c_int, T, T, P], ctypes.c_int),
+            "cp_layout_head2seq": ([ctypes.c_int, T, T, P], ctypes.c_int),
+            "cp_ring_step": ([P, ctypes.c_int, ctypes.c_int, T, T, T, T, T, P], ctypes.c_int),
+            "cp_lse_merge": ([T, T, T, T, P], ctypes.c_int),
+            "cp_device_status": ([P, P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
+            "cp_status_string": ([ctypes.c_int], ctypes.c_char_p),
+            "cp_plan_step_chunk": ([P, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                    ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
+            "cp_plan_flops": ([P, ctypes.c_int, ctypes.POINTER(ctypes.c_double)], ctypes.c_int),
+            "cp_plan_num_work_items": ([P, ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
+            "cp_version": ([], ctypes.c_char_p),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != CP_OK:
+        raise CpError(status, what)
+
+
+def tensor_desc(t: torch.Tensor) -> CpTensor:
+    """Strided-view descriptor of a device tensor (bf16 or fp32, 3-D or 4-D)."""
+    if t.dtype == torch.bfloat16:
+        dt = CP_BF16
+    elif t.dtype == torch.float32:
+        dt = CP_FP32
+    else:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    if t.dim() not in (3, 4):
+        raise ValueError("expected a 3-D or 4-D tensor")
+    d = CpTensor()
+    d.data = t.data_ptr()
+    d.dtype = dt
+    d.ndim = t.dim()
+    for i in range(t.dim()):
+        d.shape[i] = t.shape[i]
+        d.stride[i] = t.stride(i)
+    return d
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+class Plan:
+    """A cp_attn plan: validated problem geometry (host only until the first launch)."""
+
+    def __init__(self, B: int, Hq: int, Hkv: int, L: int, d: int, n_cp: int = 1, n_hp: int = 1,
+                 causal: bool = True, mode: str = "ring", split: str = "contiguous", scale: float = 0.0,
+                 wait_limit_ns: int = 0, debug_fault: int = 0):
+        self.cfg = CpConfig(B, Hq, Hkv, L, d, n_cp, n_hp, int(bool(causal)), MODES[mode], SPLITS[split],
+                            float(scale), int(wait_limit_ns), int(debug_fault))
+        self.mode = mode
+        h = ctypes.c_void_p()
+        _check(lib().cp_attn_plan(ctypes.byref(self.cfg), ctypes.byref(h)), "cp_attn_plan")
+        self._h = h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.cp_attn_plan_destroy(h)
+            self._h = None
+
+    @property
+    def scale(self) -> float:
+        return self.cfg.softmax_scale if self.cfg.softmax_scale > 0 else 1.0 / math.sqrt(self.cfg.d)
+
+    def workspace_size(self, backward: bool = False) -> int:
+        n = ctypes.c_size_t()
+        _check(lib().cp_attn_workspace_size(self._h, int(backward), ctypes.byref(n)), "cp_attn_workspace_size")
+        return n.value
+
+    def workspace(self, backward: bool = False, device=None) -> Optional[torch.Tensor]:
+        n = self.workspace_size(backward)
+        return torch.empty(max(n, 1), dtype=torch.uint8, device=device or "cuda") if n else None
+
+    def step_chunk(self, rank: int, step: int):
+        c, k = ctypes.c_int(), ctypes.c_int()
+        _check(lib().cp_plan_step_chunk(self._h, rank, step, ctypes.byref(c), ctypes.byref(k)), "cp_plan_step_chunk")
+        return c.value, k.value
+
+    def flops(self, backward: bool = False) -> float:
+        f = ctypes.c_double()
+        _check(lib().cp_plan_flops(self._h, int(backward), ctypes.byref(f)), "cp_plan_flops")
+        return f.value
+
+    def num_work_items(self) -> int:
+        n = ctypes.c_int64()
+        _check(lib().cp_plan_num_work_items(self._h, ctypes.byref(n)), "cp_plan_num_work_items")
+        return n.value
+
+    def fwd(self, q, k, v, o=None, lse=None, ws=None, stream=None):
+        """Forward; returns (o, lse).  Layouts per mode (see cp_attn.h)."""
+        c = self.cfg
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty((c.B, c.Hq, c.L), dtype=torch.float32, device=q.device)
+        if ws is None:
+            ws = self.workspace(False, q.device)
+        wptr = ws.data_ptr() if ws is not None else None
+        wlen = ws.numel() if ws is not None else 0
+        td = [tensor_desc(t) for t in (q, k, v, o, lse)]
+        _check(lib().cp_attn_fwd(self._h, *[ctypes.byref(t) for t in td], wptr, wlen, _stream(stream)),
+               "cp_attn_fwd")
+        return o, lse
+
+    def bwd(self, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, ws=None, stream=None):
+        """Backward; returns (dq, dk, dv)."""
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        if ws is None:
+            ws = self.workspace(True, q.device)
+        wptr = ws.data_ptr() if ws is not None else None
+        wlen = ws.numel() if ws is not None else 0
+        td = [tensor_desc(t) for t in (q, k, v, o, lse, dout, dq, dk, dv)]
+        _check(lib().cp_attn_bwd(self._h, *[ctypes.byref(t) for t in td], wptr, wlen, _stream(stream)),
+               "cp_attn_bwd")
+        return dq, dk, dv
+
+    def ring_step(self, rank: int, step: int, q, k, v, o_part=None, lse_part=None, stream=None):
+        """One ring step's fp32 partial (O normalised, LSE) of query chunk `rank`."""
+        c = self.cfg
+        ch = c.L // c.n_cp
+        if o_part is None:
+            o_part = torch.empty((c.B, c.Hq, ch, c.d), dtype=torch.float32, device=q.device)
+        if lse_part is None:
+            lse_part = torch.empty((c.B, c.Hq, ch), dtype=torch.float32, device=q.device)
+        td = [tensor_desc(t) for t in (q, k, v, o_part, lse_part)]
+        _check(lib().cp_ring_step(self._h, rank, step, *[ctypes.byref(t) for t in td], _stream(stream)),
+               "cp_ring_step")
+        return o_part, lse_part
+
+    def device_status(self, stream=None):
+        """Synchronise and read/clear the device status word -> (status, raw word)."""
+        w = ctypes.c_int()
+        st = lib().cp_device_status(self._h, _stream(stream), ctypes.byref(w))
+        return st, w.value
+
+
+def lse_merge(o_acc, lse_acc, o_part, lse_part, stream=None) -> None:
+    td = [tensor_desc(t) for t in (o_acc, lse_acc, o_part, lse_part)]
+    _check(lib().cp_lse_merge(*[ctypes.byref(t) for t in td], _stream(stream)), "cp_lse_merge")
+
+
+def seq2head(n_ranks: int, x, out=None, stream=None):
+    """[B, L, H, d] -> [B, H, L, d] (Ulysses all-to-all, bit-exact)."""
+    if out is None:
+        B, L, H, d = x.shape
+        out = torch.empty((B, H, L, d), dtype=x.dtype, device=x.device)
+    a, b = tensor_desc(x), tensor_desc(out)
+    _check(lib().cp_layout_seq2head(n_ranks, ctypes.byref(a), ctypes.byref(b), _stream(stream)), "cp_layout_seq2head")
+    return out
+
+
+def head2seq(n_ranks: int, x, out=None, stream=None):
+    """[B, H, L, d] -> [B, L, H, d] (inverse all-to-all, bit-exact)."""
+    if out is None:
+        B, H, L, d = x.shape
+        out = torch.empty((B, L, H, d), dtype=x.dtype, device=x.device)
+    a, b = tensor_desc(x), tensor_desc(out)
+    _check(lib().cp_layout_head2seq(n_ranks, ctypes.byref(a), ctypes.byref(b), _stream(stream)), "cp_layout_head2seq")
+    return out

@@ -1,0 +1,52 @@
+"""Named workloads: shapes of the pages' models on one GPU (synthetic, seeded inputs).
+
+  c1  tiny ring attention, MHA, d=64, L=1024, N_cp=4 (chunks of 256)
+  c2  Llama-3-8B-shaped GQA ring attention: 32 q heads / 8 KV heads, d=128, L=32768, N_cp=8,
+      inputs N(0,1)/sqrt(2)
+  c3  long-context Llama-3-8B-shaped GQA ring attention: L=212992 (208K), N_cp=16 (13312)
+  c4  Ulysses, 7B-MHA: H=32, d=128, L=131072, degree 8; sequence-major per-rank input
+  c5  2D head x context grid 4 x 4, 7B-MHA: H=32, d=128, L=65536, forward + backward
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    cfg_id: int
+    B: int
+    Hq: int
+    Hkv: int
+    L: int
+    d: int
+    n_cp: int
+    n_hp: int
+    mode: str            # ring | ulysses | 2d
+    causal: bool = True
+    input_scale: float = 1.0
+    backward: bool = False
+
+    @property
+    def seq_major(self) -> bool:
+        return self.mode != "ring"
+
+    def q_shape(self):
+        return (self.B, self.L, self.Hq, self.d) if self.seq_major else (self.B, self.Hq, self.L, self.d)
+
+    def kv_shape(self):
+        return (self.B, self.L, self.Hkv, self.d) if self.seq_major else (self.B, self.Hkv, self.L, self.d)
+
+    def fwd_flops(self) -> float:
+        pairs = self.L * (self.L + 1) / 2 if self.causal else float(self.L) ** 2
+        return 4.0 * self.B * self.Hq * self.d * pairs
+
+
+WORKLOADS = {
+    "c1": Workload("c1_tiny_ring_mha_L1024_N4", 1, 1, 4, 4, 1024, 64, 4, 1, "ring"),
+    "c2": Workload("c2_llama3_8b_gqa_L32768_N8", 2, 1, 32, 8, 32768, 128, 8, 1, "ring", input_scale=2 ** -0.5),
+    "c3": Workload("c3_llama3_8b_gqa_L212992_N16", 3, 1, 32, 8, 212992, 128, 16, 1, "ring"),
+    "c4": Workload("c4_ulysses_7b_mha_L131072_N8", 4, 1, 32, 32, 131072, 128, 8, 1, "ulysses"),
+    "c5": Workload("c5_2d_4x4_7b_mha_L65536_fwd_bwd", 5, 1, 32, 32, 65536, 128, 4, 4, "2d", backward=True),
+}

@@ -1,0 +1,192 @@
+// aux_kernels.cuh — HBM-bound kernels: Ulysses re-layout, step-wise LSE merge, and the
+// backward's D = rowsum(dO * O) preprocess and dQ fp32 -> bf16 conversion.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace cpattn {
+
+// ---- Ulysses all-to-all on one GPU -------------------------------------------------------
+// Swaps axes 1 and 2 of a [B, X, Y, d] view: out[b, y, x, :] = in[b, x, y, :].  Rows of d
+// elements are contiguous on both sides, so the copy moves whole 16-byte vectors: thread
+// groups walk the OUTPUT in order (fully sequential writes) and read 16-byte pieces of
+// 2*d-byte rows (d = 128 -> 256-byte contiguous reads).  Each thread moves kVecPerThread
+// vectors spaced one block apart, so every load of a warp is coalesced and several loads
+// per thread are in flight.  ("05. 長系列の分散学習（Context Parallelism）" §2: the
+// re-layout [D, L/N_cp] -> [H/N_cp, L]; "Ulyssesシーケンス並列化の核心" steps 2 and 4.)
+struct PermuteParams {
+  const uint4* in;
+  uint4* out;
+  long long n_vec;       // total 16-byte vectors
+  int vec_per_row;       // d * elem_bytes / 16
+  int X, Y;              // in is [B, X, Y, row]; out is [B, Y, X, row]
+  long long in_sb, in_sx, in_sy;     // strides in 16-byte vectors
+  long long out_sb, out_sy, out_sx;
+};
+
+constexpr int kPermThreads = 256;
+constexpr int kVecPerThread = 4;
+
+__global__ void __launch_bounds__(kPermThreads) permute_rows_kernel(const PermuteParams p) {
+  const long long base = static_cast<long long>(blockIdx.x) * (kPermThreads * kVecPerThread) + threadIdx.x;
+  uint4 v[kVecPerThread];
+  long long dst[kVecPerThread];
+#pragma unroll
+  for (int u = 0; u < kVecPerThread; ++u) {
+    const long long g = base + u * kPermThreads;  // index in output order (b, y, x, vec)
+    dst[u] = -1;
+    if (g < p.n_vec) {
+      long long t = g;
+      const int vec = static_cast<int>(t % p.vec_per_row);
+      t /= p.vec_per_row;
+      const int x = static_cast<int>(t % p.X);
+      t /= p.X;
+      const int y = static_cast<int>(t % p.Y);
+      const long long b = t / p.Y;
+      v[u] = __ldg(p.in + b * p.in_sb + x * p.in_sx + y * p.in_sy + vec);
+      dst[u] = b * p.out_sb + y * p.out_sy + x * p.out_sx + vec;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kVecPerThread; ++u)
+    if (dst[u] >= 0) p.out[dst[u]] = v[u];
+}
+
+// ---- step-wise LSE merge ----------------------------------------------------------------
+// (O_acc, LSE_acc) <- (O_acc, LSE_acc) (+) (O_part, LSE_part) in place ("ring attention:
+// key/value をリングで回す" step 3).  One row of d fp32 per d/4 lanes (16-byte vectors).
+struct MergeParams {
+  float* o_acc;
+  float* lse_acc;
+  const float* o_part;
+  const float* lse_part;
+  int B, H, R, d;  // rows R per (b, h)
+  long long oa_sb, oa_sh, oa_sr, la_sb, la_sh, la_sr;
+  long long op_sb, op_sh, op_sr, lp_sb, lp_sh, lp_sr;
+};
+
+__global__ void __launch_bounds__(256) lse_merge_kernel(const MergeParams p) {
+  const int lanes_per_row = p.d / 4;  // 16 or 32: a row never straddles two warps
+  const long long gthread = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = gthread / lanes_per_row;
+  const int vec = static_cast<int>(gthread % lanes_per_row);
+  const long long n_rows = static_cast<long long>(p.B) * p.H * p.R;
+  const bool live = row < n_rows;
+  float* la = nullptr;
+  float lse_out = -INFINITY;
+  if (live) {
+    const int r = static_cast<int>(row % p.R);
+    const int h = static_cast<int>((row / p.R) % p.H);
+    const int b = static_cast<int>(row / (static_cast<long long>(p.R) * p.H));
+    la = p.lse_acc + b * p.la_sb + h * p.la_sh + r * p.la_sr;
+    const float lb = p.lse_part[b * p.lp_sb + h * p.lp_sh + r * p.lp_sr];
+    const float l0 = *la;
+    const float m = fmaxf(l0, lb);
+    float4* oa = reinterpret_cast<float4*>(p.o_acc + b * p.oa_sb + h * p.oa_sh + r * p.oa_sr) + vec;
+    const float4 ob = reinterpret_cast<const float4*>(p.o_part + b * p.op_sb + h * p.op_sh + r * p.op_sr)[vec];
+    float4 out;
+    if (m == -INFINITY) {
+      out = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      const float wa = (l0 == -INFINITY) ? 0.f : expf(l0 - m);
+      const float wb = (lb == -INFINITY) ? 0.f : expf(lb - m);
+      const float inv = 1.f / (wa + wb);
+      const float ca = wa * inv, cb = wb * inv;
+      const float4 a = *oa;
+      out = make_float4(ca * a.x + cb * ob.x, ca * a.y + cb * ob.y, ca * a.z + cb * ob.z, ca * a.w + cb * ob.w);
+      lse_out = m + logf(wa + wb);
+    }
+    *oa = out;
+  }
+  // every lane of a row has read *la before its first lane overwrites it
+  __syncwarp();
+  if (live && vec == 0) *la = lse_out;
+}
+
+// ---- backward preprocess: D_i = sum_e dO_ie * O_ie ------------------------------------------
+// 16 lanes per row at d = 128 (8 at d = 64), each loading 16 bytes of dO and of O, then a
+// butterfly shuffle reduction inside the lane group.  Output D [B, H, L] fp32 (head-major).
+struct DotParams {
+  const __nv_bfloat16* o;
+  const __nv_bfloat16* dout;
+  float* D;
+  int B, H, L, d;
+  long long o_sb, o_sh, o_sl, g_sb, g_sh, g_sl;  // element strides of o and dout ([b,h,l] axes)
+  long long D_sb, D_sh, D_sl;
+};
+
+__global__ void __launch_bounds__(256) rowdot_kernel(const DotParams p) {
+  const int lpr = p.d / 8;  // lanes per row (power of two)
+  const long long gthread = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = gthread / lpr;
+  const int vec = static_cast<int>(gthread % lpr);
+  const long long n_rows = static_cast<long long>(p.B) * p.H * p.L;
+  const bool live = row < n_rows;
+  float acc = 0.f;
+  int b = 0, h = 0, l = 0;
+  if (live) {
+    l = static_cast<int>(row % p.L);
+    h = static_cast<int>((row / p.L) % p.H);
+    b = static_cast<int>(row / (static_cast<long long>(p.L) * p.H));
+    const uint4 a = reinterpret_cast<const uint4*>(p.o + b * p.o_sb + h * p.o_sh + l * p.o_sl)[vec];
+    const uint4 g = reinterpret_cast<const uint4*>(p.dout + b * p.g_sb + h * p.g_sh + l * p.g_sl)[vec];
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(a2[e]);
+      const float2 y = __bfloat1622float2(g2[e]);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
+    }
+  }
+  for (int off = lpr >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (live && vec == 0) p.D[b * p.D_sb + h * p.D_sh + l * p.D_sl] = acc;
+}
+
+// ---- dQ accumulator (fp32, already scaled) -> bf16 output ------------------------------------
+struct CastParams {
+  const float* src;      // contiguous [B, H, L, d]
+  __nv_bfloat16* dst;
+  int B, H, L, d;
+  long long d_sb, d_sh, d_sl;
+};
+
+__global__ void __launch_bounds__(256) cast_bf16_kernel(const CastParams p) {
+  const long long n4 = static_cast<long long>(p.B) * p.H * p.L * p.d / 4;
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const long long e = i * 4;
+  const int c = static_cast<int>(e % p.d);
+  long long t = e / p.d;
+  const int l = static_cast<int>(t % p.L);
+  t /= p.L;
+  const int h = static_cast<int>(t % p.H);
+  const int b = static_cast<int>(t / p.H);
+  const float4 v = reinterpret_cast<const float4*>(p.src)[i];
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 packed;
+  packed.x = *reinterpret_cast<uint32_t*>(&lo);
+  packed.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(p.dst + b * p.d_sb + h * p.d_sh + l * p.d_sl + c) = packed;
+}
+
+// ---- fill a step-wise partial with the merge identity (O = 0, LSE = -inf) -------------------
+__global__ void fill_identity_kernel(float* o, float* lse, int B, int H, int R, int d, long long o_sb,
+                                     long long o_sh, long long o_sr, long long l_sb, long long l_sh,
+                                     long long l_sr) {
+  const long long n = static_cast<long long>(B) * H * R * d;
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int c = static_cast<int>(i % d);
+  long long t = i / d;
+  const int r = static_cast<int>(t % R);
+  t /= R;
+  const int h = static_cast<int>(t % H);
+  const int b = static_cast<int>(t / H);
+  o[b * o_sb + h * o_sh + r * o_sr + c] = 0.f;
+  if (c == 0) lse[b * l_sb + h * l_sh + r * l_sr] = -INFINITY;
+}
+
+}  // namespace cpattn

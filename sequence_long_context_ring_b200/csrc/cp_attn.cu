@@ -1,0 +1,524 @@
+// cp_attn.cu — host side of libcpattn.so: plan construction and validation, TMA tensor-map
+// encoding, workspace carving, and the launches behind the C ABI declared in cp_attn.h.
+#include "cp_attn.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <new>
+
+#include "aux_kernels.cuh"
+#include "bwd_kernel.cuh"
+#include "fwd_kernel.cuh"
+
+using namespace cpattn;
+
+struct cp_plan {
+  cp_attn_config_t cfg;
+  int G;
+  float scale;
+  mutable std::mutex mu;
+  mutable std::map<int, int*> status_words;  // per device ordinal
+};
+
+namespace {
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int elem_bytes(cp_dtype_t t) { return t == CP_BF16 ? 2 : 4; }
+
+// Check a 4-D data tensor: dtype, exact shape, innermost stride 1, other strides x element
+// size multiples of 16 bytes, 16-byte aligned base (the TMA / 128-bit vector rules).
+cp_status_t check4(const cp_tensor_t* t, cp_dtype_t dt, int64_t s0, int64_t s1, int64_t s2, int64_t s3) {
+  if (!t || !t->data) return CP_ERR_INVALID_ARG;
+  if (t->ndim != 4 || t->dtype != dt) return CP_ERR_INVALID_ARG;
+  if (t->shape[0] != s0 || t->shape[1] != s1 || t->shape[2] != s2 || t->shape[3] != s3) return CP_ERR_INVALID_ARG;
+  if (t->stride[3] != 1) return CP_ERR_ALIGNMENT;
+  const int eb = elem_bytes(dt);
+  for (int i = 0; i < 3; ++i)
+    if (t->stride[i] <= 0 || (t->stride[i] * eb) % 16 != 0) return CP_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(t->data) % 16 != 0) return CP_ERR_ALIGNMENT;
+  return CP_OK;
+}
+
+// Check a 3-D fp32 row-statistics tensor (LSE / D): exact shape, 4-byte aligned, any strides.
+cp_status_t check3(const cp_tensor_t* t, int64_t s0, int64_t s1, int64_t s2) {
+  if (!t || !t->data) return CP_ERR_INVALID_ARG;
+  if (t->ndim != 3 || t->dtype != CP_FP32) return CP_ERR_INVALID_ARG;
+  if (t->shape[0] != s0 || t->shape[1] != s1 || t->shape[2] != s2) return CP_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (t->stride[i] < 0) return CP_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(t->data) % 4 != 0) return CP_ERR_ALIGNMENT;
+  return CP_OK;
+}
+
+#define CP_TRY(expr)                 \
+  do {                               \
+    cp_status_t st__ = (expr);       \
+    if (st__ != CP_OK) return st__;  \
+  } while (0)
+
+// ---- device status word -----------------------------------------------------------------
+int* status_word(const cp_plan_t* plan, cp_status_t* err) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    *err = CP_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> g(plan->mu);
+  auto it = plan->status_words.find(dev);
+  if (it != plan->status_words.end()) return it->second;
+  int* w = nullptr;
+  if (cudaMalloc(&w, sizeof(int)) != cudaSuccess || cudaMemset(w, 0, sizeof(int)) != cudaSuccess) {
+    *err = CP_ERR_CUDA;
+    return nullptr;
+  }
+  plan->status_words[dev] = w;
+  return w;
+}
+
+// ---- TMA tensor maps --------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a bf16 view [B, H, L, d] (strides in elements, innermost 1): dimensions
+// (d, L, H, B) with 64 x 128 x 1 x 1 boxes, 128-byte swizzle, zero fill out of bounds.
+cp_status_t make_map_bhld(CUtensorMap* m, const void* base, int64_t B, int64_t H, int64_t L, int64_t d,
+                          int64_t sB, int64_t sH, int64_t sL) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CP_ERR_CUDA;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)(sL * 2), (cuuint64_t)(sH * 2), (cuuint64_t)(sB * 2)};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CP_OK : CP_ERR_CUDA;
+}
+
+// A [B, H, L, d] view given either directly (head-major) or as the plain pointer of a
+// contiguous head-major workspace buffer.
+struct View {
+  const void* data;
+  int64_t B, H, L, d, sB, sH, sL;
+};
+View view_of(const cp_tensor_t* t) {
+  return View{t->data, t->shape[0], t->shape[1], t->shape[2], t->shape[3], t->stride[0], t->stride[1], t->stride[2]};
+}
+View contiguous_view(const void* p, int64_t B, int64_t H, int64_t L, int64_t d) {
+  return View{p, B, H, L, d, H * L * d, L * d, d};
+}
+
+template <int D>
+cp_status_t launch_fwd_d(const FwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         int64_t grid, cudaStream_t s) {
+  const size_t smem = fwd_smem_bytes(D);
+  if (cudaFuncSetAttribute(ring_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return CP_ERR_CUDA;
+  ring_fwd_kernel<D><<<(unsigned)grid, kFwdThreads, smem, s>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+struct FwdOut {
+  void* o;
+  int64_t o_sb, o_sh, o_sl;
+  int out_fp32;
+  float* lse;
+  int64_t l_sb, l_sh, l_sl;
+};
+
+// Work decomposition of the fused forward for a ring of n_chunks over [B, H, L, d].
+void fill_geometry(const cp_plan_t* plan, int n_chunks, FwdParams& p) {
+  const cp_attn_config_t& c = plan->cfg;
+  p.B = c.B;
+  p.Hq = c.Hq;
+  p.Hkv = c.Hkv;
+  p.L = c.L;
+  p.d = c.d;
+  p.G = plan->G;
+  p.n_chunks = n_chunks;
+  p.chunk_len = c.L / n_chunks;
+  p.tiles_per_chunk = (p.chunk_len + kBN - 1) / kBN;
+  p.pair_heads = (plan->G % 2 == 0) ? 1 : 0;
+  p.pos_per_chunk = p.pair_heads ? p.tiles_per_chunk : (p.tiles_per_chunk + 1) / 2;
+  p.n_inner = p.pair_heads ? c.B * c.Hkv * (plan->G / 2) : c.B * c.Hq;
+  p.causal = c.causal ? 1 : 0;
+  p.scale_log2 = static_cast<float>(static_cast<double>(plan->scale) * 1.4426950408889634);
+  p.step_rank = -1;
+  p.step_chunk = 0;
+  p.out_row_base = 0;
+  p.wait_limit_ns = c.wait_limit_ns ? c.wait_limit_ns : kDefaultWaitLimitNs;
+  p.debug_fault = c.debug_fault;
+}
+
+cp_status_t run_fwd_kernel(const cp_plan_t* plan, FwdParams& p, const View& q, const View& k, const View& v,
+                           const FwdOut& out, int64_t grid, cudaStream_t s) {
+  cp_status_t err = CP_OK;
+  int* sw = status_word(plan, &err);
+  if (!sw) return err;
+  p.o = out.o;
+  p.o_sb = out.o_sb;
+  p.o_sh = out.o_sh;
+  p.o_sl = out.o_sl;
+  p.out_fp32 = out.out_fp32;
+  p.lse = out.lse;
+  p.l_sb = out.l_sb;
+  p.l_sh = out.l_sh;
+  p.l_sl = out.l_sl;
+  p.status = sw;
+  CUtensorMap mq, mk, mv;
+  CP_TRY(make_map_bhld(&mq, q.data, q.B, q.H, q.L, q.d, q.sB, q.sH, q.sL));
+  CP_TRY(make_map_bhld(&mk, k.data, k.B, k.H, k.L, k.d, k.sB, k.sH, k.sL));
+  CP_TRY(make_map_bhld(&mv, v.data, v.B, v.H, v.L, v.d, v.sB, v.sH, v.sL));
+  if (grid <= 0) return CP_OK;
+  if (p.d == 128) return launch_fwd_d<128>(p, mq, mk, mv, grid, s);
+  return launch_fwd_d<64>(p, mq, mk, mv, grid, s);
+}
+
+// ---- permute ------------------------------------------------------------------------------
+// out[b, y, x, :] = in[b, x, y, :] for in [B, X, Y, d] (element strides given per axis).
+cp_status_t launch_permute(const void* in, void* out, int64_t B, int64_t X, int64_t Y, int64_t d, int eb,
+                           const int64_t in_str[3], const int64_t out_str_yx[3], cudaStream_t s) {
+  const int64_t row_bytes = d * eb;
+  if (row_bytes % 16 != 0) return CP_ERR_ALIGNMENT;
+  PermuteParams p;
+  p.in = static_cast<const uint4*>(in);
+  p.out = static_cast<uint4*>(out);
+  p.vec_per_row = static_cast<int>(row_bytes / 16);
+  p.X = static_cast<int>(X);
+  p.Y = static_cast<int>(Y);
+  p.n_vec = B * X * Y * p.vec_per_row;
+  const int64_t per = 16 / eb;
+  p.in_sb = in_str[0] / per;
+  p.in_sx = in_str[1] / per;
+  p.in_sy = in_str[2] / per;
+  p.out_sb = out_str_yx[0] / per;
+  p.out_sy = out_str_yx[1] / per;
+  p.out_sx = out_str_yx[2] / per;
+  if (p.n_vec == 0) return CP_OK;
+  const int64_t per_block = kPermThreads * kVecPerThread;
+  const int64_t grid = (p.n_vec + per_block - 1) / per_block;
+  permute_rows_kernel<<<(unsigned)grid, kPermThreads, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+// seq-major [B, L, H, d] tensor -> contiguous head-major buffer [B, H, L, d]
+cp_status_t seq_to_head_buf(const cp_tensor_t* in, void* buf, cudaStream_t s) {
+  const int64_t B = in->shape[0], L = in->shape[1], H = in->shape[2], d = in->shape[3];
+  const int64_t in_str[3] = {in->stride[0], in->stride[1], in->stride[2]};
+  const int64_t out_str[3] = {H * L * d, L * d, d};  // (b, y=h, x=l)
+  return launch_permute(in->data, buf, B, L, H, d, elem_bytes(in->dtype), in_str, out_str, s);
+}
+// contiguous head-major buffer [B, H, L, d] -> seq-major tensor [B, L, H, d]
+cp_status_t head_buf_to_seq(const void* buf, cp_tensor_t* out, cudaStream_t s) {
+  const int64_t B = out->shape[0], L = out->shape[1], H = out->shape[2], d = out->shape[3];
+  const int64_t in_str[3] = {H * L * d, L * d, d};                      // (b, x=h, y=l)
+  const int64_t out_str[3] = {out->stride[0], out->stride[1], out->stride[2]};  // (b, y=l, x=h)
+  return launch_permute(buf, out->data, B, H, L, d, elem_bytes(out->dtype), in_str, out_str, s);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_tensor_t* k, const cp_tensor_t* v,
+                         const cp_tensor_t* o, const cp_tensor_t* lse, const cp_tensor_t* dout, cp_tensor_t* dq,
+                         cp_tensor_t* dk, cp_tensor_t* dv, void* ws, size_t ws_bytes, void* stream) {
+  (void)q; (void)k; (void)v; (void)o; (void)lse; (void)dout; (void)dq; (void)dk; (void)dv;
+  (void)ws; (void)ws_bytes; (void)stream;
+  if (!plan) return CP_ERR_INVALID_ARG;
+  return CP_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+// =====================================================================================
+extern "C" {
+
+const char* cp_version(void) { return "cpattn 0.1 (sm_100a tcgen05)"; }
+
+const char* cp_status_string(cp_status_t s) {
+  switch (s) {
+    case CP_OK: return "ok";
+    case CP_ERR_INVALID_ARG: return "invalid argument";
+    case CP_ERR_UNSUPPORTED: return "unsupported configuration";
+    case CP_ERR_ALIGNMENT: return "alignment or stride violation";
+    case CP_ERR_WORKSPACE: return "workspace missing or too small";
+    case CP_ERR_CUDA: return "CUDA error";
+    case CP_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+cp_status_t cp_attn_plan(const cp_attn_config_t* cfg, cp_plan_t** out) {
+  if (!cfg || !out) return CP_ERR_INVALID_ARG;
+  const cp_attn_config_t& c = *cfg;
+  if (c.B < 1 || c.Hq < 1 || c.Hkv < 1 || c.L < 1 || c.d < 1 || c.n_cp < 1 || c.n_hp < 1) return CP_ERR_INVALID_ARG;
+  if (c.Hq % c.Hkv != 0) return CP_ERR_INVALID_ARG;
+  if (c.causal != 0 && c.causal != 1) return CP_ERR_INVALID_ARG;
+  if (!(c.softmax_scale >= 0.f) || std::isinf(c.softmax_scale)) return CP_ERR_INVALID_ARG;
+  if (c.split == CP_SPLIT_ZIGZAG) return CP_ERR_UNSUPPORTED;
+  if (c.split != CP_SPLIT_CONTIGUOUS) return CP_ERR_INVALID_ARG;
+  switch (c.mode) {
+    case CP_MODE_RING:
+      if (c.n_hp != 1 || c.L % c.n_cp != 0) return CP_ERR_INVALID_ARG;
+      break;
+    case CP_MODE_ULYSSES:
+      if (c.n_hp != 1 || c.L % c.n_cp != 0) return CP_ERR_INVALID_ARG;
+      if (c.Hq % c.n_cp != 0 || c.Hkv % c.n_cp != 0) return CP_ERR_INVALID_ARG;
+      break;
+    case CP_MODE_2D:
+      if ((int64_t)c.n_hp * c.n_cp <= 0 || c.L % (c.n_hp * c.n_cp) != 0) return CP_ERR_INVALID_ARG;
+      if (c.Hq % c.n_hp != 0 || c.Hkv % c.n_hp != 0) return CP_ERR_INVALID_ARG;
+      break;
+    default:
+      return CP_ERR_INVALID_ARG;
+  }
+  if (c.d != 64 && c.d != 128) return CP_ERR_UNSUPPORTED;
+  if (c.debug_fault < 0 || c.debug_fault > 1) return CP_ERR_INVALID_ARG;
+  cp_plan_t* p = new (std::nothrow) cp_plan_t();
+  if (!p) return CP_ERR_INVALID_ARG;
+  p->cfg = c;
+  p->G = c.Hq / c.Hkv;
+  p->scale = c.softmax_scale > 0.f ? c.softmax_scale : static_cast<float>(1.0 / std::sqrt((double)c.d));
+  *out = p;
+  return CP_OK;
+}
+
+void cp_attn_plan_destroy(cp_plan_t* plan) {
+  if (!plan) return;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  for (auto& kv : plan->status_words) {
+    if (cudaSetDevice(kv.first) == cudaSuccess) cudaFree(kv.second);
+  }
+  if (prev >= 0) cudaSetDevice(prev);
+  delete plan;
+}
+
+cp_status_t cp_attn_workspace_size(const cp_plan_t* plan, int backward, size_t* bytes) {
+  if (!plan || !bytes) return CP_ERR_INVALID_ARG;
+  const cp_attn_config_t& c = plan->cfg;
+  const size_t nq = (size_t)c.B * c.Hq * c.L * c.d, nkv = (size_t)c.B * c.Hkv * c.L * c.d;
+  const size_t nrow = (size_t)c.B * c.Hq * c.L;
+  const bool seq_major = c.mode != CP_MODE_RING;
+  size_t ws = 0;
+  if (!backward) {
+    if (seq_major) ws = 2 * align256(nq * 2) + 2 * align256(nkv * 2);
+  } else {
+    ws = align256(nq * 4) + align256(nrow * 4) + bwd_workspace_extra(c.B, c.Hq, c.Hkv, c.L, c.d);
+    if (seq_major) ws += 3 * align256(nq * 2) + 4 * align256(nkv * 2);  // q, do, dq ; k, v, dk, dv
+  }
+  *bytes = ws;
+  return CP_OK;
+}
+
+cp_status_t cp_attn_fwd(const cp_plan_t* plan, const cp_tensor_t* q, const cp_tensor_t* k, const cp_tensor_t* v,
+                        cp_tensor_t* o, cp_tensor_t* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!plan) return CP_ERR_INVALID_ARG;
+  const cp_attn_config_t& c = plan->cfg;
+  const cudaStream_t s = as_stream(stream);
+  CP_TRY(check3(lse, c.B, c.Hq, c.L));
+  FwdParams p{};
+  if (c.mode == CP_MODE_RING) {
+    CP_TRY(check4(q, CP_BF16, c.B, c.Hq, c.L, c.d));
+    CP_TRY(check4(k, CP_BF16, c.B, c.Hkv, c.L, c.d));
+    CP_TRY(check4(v, CP_BF16, c.B, c.Hkv, c.L, c.d));
+    CP_TRY(check4(o, CP_BF16, c.B, c.Hq, c.L, c.d));
+    fill_geometry(plan, c.n_cp, p);
+    const int64_t grid = (int64_t)p.n_chunks * p.pos_per_chunk * p.n_inner;
+    FwdOut out{o->data, o->stride[0], o->stride[1], o->stride[2], 0, static_cast<float*>(lse->data),
+               lse->stride[0], lse->stride[1], lse->stride[2]};
+    return run_fwd_kernel(plan, p, view_of(q), view_of(k), view_of(v), out, grid, s);
+  }
+  // ULYSSES / TWO_D: sequence-major in and out, head-major in the workspace.
+  CP_TRY(check4(q, CP_BF16, c.B, c.L, c.Hq, c.d));
+  CP_TRY(check4(k, CP_BF16, c.B, c.L, c.Hkv, c.d));
+  CP_TRY(check4(v, CP_BF16, c.B, c.L, c.Hkv, c.d));
+  CP_TRY(check4(o, CP_BF16, c.B, c.L, c.Hq, c.d));
+  size_t need = 0;
+  cp_attn_workspace_size(plan, 0, &need);
+  if (!ws || ws_bytes < need) return CP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return CP_ERR_ALIGNMENT;
+  const size_t nq = (size_t)c.B * c.Hq * c.L * c.d, nkv = (size_t)c.B * c.Hkv * c.L * c.d;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  void* qh = w;
+  w += align256(nq * 2);
+  void* kh = w;
+  w += align256(nkv * 2);
+  void* vh = w;
+  w += align256(nkv * 2);
+  void* oh = w;
+  // step 2 of the Ulysses flow (head-group all-to-all for 2D): seq -> head
+  CP_TRY(seq_to_head_buf(q, qh, s));
+  CP_TRY(seq_to_head_buf(k, kh, s));
+  CP_TRY(seq_to_head_buf(v, vh, s));
+  // step 3: attention per head group (Ulysses: one chunk = full sequence; 2D: ring over n_cp)
+  fill_geometry(plan, c.mode == CP_MODE_ULYSSES ? 1 : c.n_cp, p);
+  const int64_t grid = (int64_t)p.n_chunks * p.pos_per_chunk * p.n_inner;
+  FwdOut out{oh, (int64_t)c.Hq * c.L * c.d, (int64_t)c.L * c.d, c.d, 0, static_cast<float*>(lse->data),
+             lse->stride[0], lse->stride[1], lse->stride[2]};
+  CP_TRY(run_fwd_kernel(plan, p, contiguous_view(qh, c.B, c.Hq, c.L, c.d), contiguous_view(kh, c.B, c.Hkv, c.L, c.d),
+                        contiguous_view(vh, c.B, c.Hkv, c.L, c.d), out, grid, s));
+  // step 4: head -> seq
+  return head_buf_to_seq(oh, o, s);
+}
+
+cp_status_t cp_ring_step(const cp_plan_t* plan, int rank, int step, const cp_tensor_t* q, const cp_tensor_t* k,
+                         const cp_tensor_t* v, cp_tensor_t* o_part, cp_tensor_t* lse_part, void* stream) {
+  if (!plan) return CP_ERR_INVALID_ARG;
+  const cp_attn_config_t& c = plan->cfg;
+  if (c.mode != CP_MODE_RING) return CP_ERR_INVALID_ARG;
+  const int N = c.n_cp;
+  if (rank < 0 || rank >= N || step < 0 || step >= N) return CP_ERR_INVALID_ARG;
+  const int ch = c.L / N;
+  CP_TRY(check4(q, CP_BF16, c.B, c.Hq, c.L, c.d));
+  CP_TRY(check4(k, CP_BF16, c.B, c.Hkv, c.L, c.d));
+  CP_TRY(check4(v, CP_BF16, c.B, c.Hkv, c.L, c.d));
+  CP_TRY(check4(o_part, CP_FP32, c.B, c.Hq, ch, c.d));
+  CP_TRY(check3(lse_part, c.B, c.Hq, ch));
+  const cudaStream_t s = as_stream(stream);
+  const int j = ((rank - step) % N + N) % N;
+  if (c.causal && j > rank) {
+    const int64_t n = (int64_t)c.B * c.Hq * ch * c.d;
+    fill_identity_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+        static_cast<float*>(o_part->data), static_cast<float*>(lse_part->data), c.B, c.Hq, ch, c.d,
+        o_part->stride[0], o_part->stride[1], o_part->stride[2], lse_part->stride[0], lse_part->stride[1],
+        lse_part->stride[2]);
+    return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+  }
+  FwdParams p{};
+  fill_geometry(plan, N, p);
+  p.step_rank = rank;
+  p.step_chunk = j;
+  p.out_row_base = rank * ch;
+  const int64_t grid = (int64_t)p.pos_per_chunk * p.n_inner;
+  FwdOut out{o_part->data, o_part->stride[0], o_part->stride[1], o_part->stride[2], 1,
+             static_cast<float*>(lse_part->data), lse_part->stride[0], lse_part->stride[1], lse_part->stride[2]};
+  return run_fwd_kernel(plan, p, view_of(q), view_of(k), view_of(v), out, grid, s);
+}
+
+cp_status_t cp_lse_merge(cp_tensor_t* o_acc, cp_tensor_t* lse_acc, const cp_tensor_t* o_part,
+                         const cp_tensor_t* lse_part, void* stream) {
+  if (!o_acc) return CP_ERR_INVALID_ARG;
+  const int64_t B = o_acc->shape[0], H = o_acc->shape[1], R = o_acc->shape[2], d = o_acc->shape[3];
+  if (d != 64 && d != 128) return CP_ERR_UNSUPPORTED;
+  CP_TRY(check4(o_acc, CP_FP32, B, H, R, d));
+  CP_TRY(check4(o_part, CP_FP32, B, H, R, d));
+  CP_TRY(check3(lse_acc, B, H, R));
+  CP_TRY(check3(lse_part, B, H, R));
+  MergeParams p{static_cast<float*>(o_acc->data), static_cast<float*>(lse_acc->data),
+                static_cast<const float*>(o_part->data), static_cast<const float*>(lse_part->data),
+                (int)B, (int)H, (int)R, (int)d,
+                o_acc->stride[0], o_acc->stride[1], o_acc->stride[2],
+                lse_acc->stride[0], lse_acc->stride[1], lse_acc->stride[2],
+                o_part->stride[0], o_part->stride[1], o_part->stride[2],
+                lse_part->stride[0], lse_part->stride[1], lse_part->stride[2]};
+  const int64_t threads = B * H * R * (d / 4);
+  if (threads == 0) return CP_OK;
+  lse_merge_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, as_stream(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status_t cp_layout_seq2head(int n_ranks, const cp_tensor_t* in, cp_tensor_t* out, void* stream) {
+  if (!in || !out || n_ranks < 1) return CP_ERR_INVALID_ARG;
+  const int64_t B = in->shape[0], L = in->shape[1], H = in->shape[2], d = in->shape[3];
+  if (in->dtype != out->dtype) return CP_ERR_INVALID_ARG;
+  CP_TRY(check4(in, in->dtype, B, L, H, d));
+  CP_TRY(check4(out, out->dtype, B, H, L, d));
+  if (H % n_ranks != 0 || L % n_ranks != 0) return CP_ERR_INVALID_ARG;
+  const int64_t in_str[3] = {in->stride[0], in->stride[1], in->stride[2]};
+  const int64_t out_str[3] = {out->stride[0], out->stride[1], out->stride[2]};  // (b, y=h, x=l)
+  return launch_permute(in->data, out->data, B, L, H, d, elem_bytes(in->dtype), in_str, out_str, as_stream(stream));
+}
+
+cp_status_t cp_layout_head2seq(int n_ranks, const cp_tensor_t* in, cp_tensor_t* out, void* stream) {
+  if (!in || !out || n_ranks < 1) return CP_ERR_INVALID_ARG;
+  const int64_t B = in->shape[0], H = in->shape[1], L = in->shape[2], d = in->shape[3];
+  if (in->dtype != out->dtype) return CP_ERR_INVALID_ARG;
+  CP_TRY(check4(in, in->dtype, B, H, L, d));
+  CP_TRY(check4(out, out->dtype, B, L, H, d));
+  if (H % n_ranks != 0 || L % n_ranks != 0) return CP_ERR_INVALID_ARG;
+  const int64_t in_str[3] = {in->stride[0], in->stride[1], in->stride[2]};
+  const int64_t out_str[3] = {out->stride[0], out->stride[1], out->stride[2]};  // (b, y=l, x=h)
+  return launch_permute(in->data, out->data, B, H, L, d, elem_bytes(in->dtype), in_str, out_str, as_stream(stream));
+}
+
+cp_status_t cp_device_status(const cp_plan_t* plan, void* stream, int* detail) {
+  if (!plan) return CP_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return CP_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CP_ERR_CUDA;
+  int* w = nullptr;
+  {
+    std::lock_guard<std::mutex> g(plan->mu);
+    auto it = plan->status_words.find(dev);
+    if (it != plan->status_words.end()) w = it->second;
+  }
+  int word = 0;
+  if (w) {
+    if (cudaMemcpy(&word, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return CP_ERR_CUDA;
+    if (word != 0 && cudaMemset(w, 0, sizeof(int)) != cudaSuccess) return CP_ERR_CUDA;
+  }
+  if (detail) *detail = word;
+  if (word == 0) return CP_OK;
+  return static_cast<cp_status_t>(-(word & 0xff));
+}
+
+cp_status_t cp_plan_step_chunk(const cp_plan_t* plan, int rank, int step, int* chunk, int* kind) {
+  if (!plan || !chunk || !kind) return CP_ERR_INVALID_ARG;
+  const cp_attn_config_t& c = plan->cfg;
+  const int N = c.mode == CP_MODE_ULYSSES ? 1 : c.n_cp;
+  if (rank < 0 || rank >= N || step < 0 || step >= N) return CP_ERR_INVALID_ARG;
+  const int j = ((rank - step) % N + N) % N;
+  *chunk = j;
+  *kind = !c.causal ? 1 : (j > rank ? 0 : (j == rank ? 2 : 1));
+  return CP_OK;
+}
+
+cp_status_t cp_plan_flops(const cp_plan_t* plan, int backward, double* flops) {
+  if (!plan || !flops) return CP_ERR_INVALID_ARG;
+  const cp_attn_config_t& c = plan->cfg;
+  const double L = c.L;
+  const double pairs = c.causal ? L * (L + 1) / 2.0 : L * L;
+  const double fwd = 4.0 * c.B * c.Hq * c.d * pairs;
+  *flops = backward ? 2.5 * fwd : fwd;
+  return CP_OK;
+}
+
+cp_status_t cp_plan_num_work_items(const cp_plan_t* plan, int64_t* n) {
+  if (!plan || !n) return CP_ERR_INVALID_ARG;
+  const cp_attn_config_t& c = plan->cfg;
+  FwdParams p{};
+  fill_geometry(plan, c.mode == CP_MODE_ULYSSES ? 1 : c.n_cp, p);
+  *n = (int64_t)p.n_chunks * p.pos_per_chunk * p.n_inner;
+  return CP_OK;
+}
+
+cp_status_t cp_attn_bwd(const cp_plan_t* plan, const cp_tensor_t* q, const cp_tensor_t* k, const cp_tensor_t* v,
+                        const cp_tensor_t* o, const cp_tensor_t* lse, const cp_tensor_t* dout, cp_tensor_t* dq,
+                        cp_tensor_t* dk, cp_tensor_t* dv, void* ws, size_t ws_bytes, void* stream) {
+  return run_backward(plan, q, k, v, o, lse, dout, dq, dk, dv, ws, ws_bytes, stream);
+}
+
+}  // extern "C"

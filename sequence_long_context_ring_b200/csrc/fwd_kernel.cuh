@@ -1,0 +1,469 @@
+// fwd_kernel.cuh — fused ring-attention forward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// What it computes ("ring attention: key/value をリングで回す", steps 1-4, in "05. 長系列の分散
+// 学習（Context Parallelism）"): virtual rank r keeps its query chunk; at ring step s it holds
+// KV chunk j = (r - s) mod N and computes the partial attention of its queries against that
+// chunk; the partials are combined by the online-softmax (LSE) merge.  Chunks wholly above
+// the causal diagonal (j > r) are skipped; the diagonal chunk (j = r) is masked key <= query.
+//
+// One CTA owns two 128-row query tiles (A, B) that stream the same KV tiles:
+//   * GQA (G even): two query heads of one KV group at the same rows;
+//   * otherwise:    two consecutive 128-row tiles of one head inside one chunk.
+// The KV tiles are visited in ring order: the diagonal chunk r first, then r-1, ..., 0.
+// Within a work item the running (max, sum, O) state is carried across tiles, so the merge
+// of a finished chunk's partial into the accumulator happens at every chunk boundary as the
+// same rescale-and-add that joins two tiles: (O, LSE) (+) (O', LSE') with weights e^(LSE-m).
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax for tile A (thread t <-> query row t <-> TMEM lane t)
+//   warps 4-7  softmax for tile B
+//   warp  8    TMA producer: Q tiles once, then K_i, V_i into a 4-stage shared-memory ring
+//   warp  9    MMA issuer (one thread): S = Q K^T into TMEM, O += P V with P read from TMEM
+// TMEM (512 columns x 128 lanes x 32 bit): S_A [0,128) O_A [128,256) S_B [256,384)
+// O_B [384,512).  P (bf16, packed two per column) overwrites the first 64 columns of S.
+//
+// Every wait is bounded (WaitCtl): on expiry the kernel records CP_ERR_TIMEOUT with the wait
+// site in the status word, drains its in-flight copies and MMAs, frees TMEM and returns.
+#pragma once
+#include "sm100.cuh"
+
+namespace cpattn {
+
+constexpr int kBM = 128;       // query rows per tile
+constexpr int kBN = 128;       // keys per KV tile
+constexpr int kStages = 4;     // shared-memory ring, one K or V tile per stage
+constexpr int kFwdThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: skip the O rescale below 2^8 growth
+
+enum WaitSite : int {
+  kSiteLoadEmpty = 1, kSiteMmaQ = 2, kSiteMmaKV = 3, kSiteMmaP = 4,
+  kSiteSoftS = 5, kSiteSoftO = 6, kSiteDrain = 7,
+};
+
+struct FwdParams {
+  int B, Hq, Hkv, L, d, G;
+  int n_chunks, chunk_len;   // ring size N and chunk length c
+  int tiles_per_chunk;       // ceil(c / 128)
+  int pos_per_chunk;         // work-item positions along the query axis of one chunk
+  int pair_heads;            // 1: A/B are heads (2p, 2p+1) of a KV group; 0: consecutive tiles
+  int n_inner;               // work items per query position
+  int causal;
+  float scale_log2;          // softmax scale * log2(e)
+  int step_rank;             // -1: fused over all ranks and steps; else one (rank, chunk) step
+  int step_chunk;
+  int out_row_base;          // subtracted from the global row when writing o / lse
+  void* o;                   // bf16 or fp32 output, [B, Hq, rows, d]
+  long long o_sb, o_sh, o_sl;
+  int out_fp32;
+  float* lse;                // [B, Hq, rows]
+  long long l_sb, l_sh, l_sl;
+  int* status;
+  unsigned long long wait_limit_ns;
+  int debug_fault;
+};
+
+struct Item {
+  int b, g, headA, headB, rowA, rowB, r, q_end, n_tiles, n_diag;
+};
+
+__device__ __forceinline__ Item decode_item(const FwdParams& p) {
+  Item it;
+  const int idx = blockIdx.x;
+  const int pos = idx / p.n_inner;
+  const int inner = idx - pos * p.n_inner;
+  int qpos;
+  if (p.step_rank >= 0) {
+    it.r = p.step_rank;
+    qpos = p.pos_per_chunk - 1 - pos;
+  } else {
+    // longest-first: last chunk, last query tiles first (the causal work grows with the row)
+    it.r = p.n_chunks - 1 - pos / p.pos_per_chunk;
+    qpos = p.pos_per_chunk - 1 - pos % p.pos_per_chunk;
+  }
+  const int c0 = it.r * p.chunk_len;
+  it.q_end = min(c0 + p.chunk_len, p.L);
+  int last;  // last valid query row of the item
+  if (p.pair_heads) {
+    const int half = p.G >> 1;
+    it.b = inner / (p.Hkv * half);
+    const int rem = inner - it.b * (p.Hkv * half);
+    it.g = rem / half;
+    const int pr = rem - it.g * half;
+    it.headA = it.g * p.G + 2 * pr;
+    it.headB = it.headA + 1;
+    it.rowA = c0 + qpos * kBM;
+    it.rowB = it.rowA;
+    last = min(it.rowA + kBM, it.q_end) - 1;
+  } else {
+    it.b = inner / p.Hq;
+    it.headA = inner - it.b * p.Hq;
+    it.headB = it.headA;
+    it.g = it.headA / p.G;
+    it.rowA = c0 + (2 * qpos) * kBM;
+    it.rowB = it.rowA + kBM;
+    last = min(it.rowB + kBM, it.q_end) - 1;
+  }
+  it.n_diag = (last - c0) / kBN + 1;
+  if (p.step_rank >= 0) {
+    it.n_tiles = (p.causal && p.step_chunk == it.r) ? it.n_diag : p.tiles_per_chunk;
+  } else if (p.causal) {
+    it.n_tiles = it.n_diag + it.r * p.tiles_per_chunk;
+  } else {
+    it.n_tiles = p.n_chunks * p.tiles_per_chunk;
+  }
+  return it;
+}
+
+// i-th KV tile of the item in ring visit order -> first key row and end of its chunk.
+__device__ __forceinline__ void kv_tile(const FwdParams& p, const Item& it, int i, int& kv0, int& kv_end) {
+  int j, tt;
+  if (p.step_rank >= 0) {
+    j = p.step_chunk;
+    tt = i;
+  } else if (p.causal) {
+    if (i < it.n_diag) {
+      j = it.r;
+      tt = i;
+    } else {
+      const int i2 = i - it.n_diag;
+      const int q = i2 / p.tiles_per_chunk;
+      j = it.r - 1 - q;
+      tt = i2 - q * p.tiles_per_chunk;
+    }
+  } else {
+    const int s = i / p.tiles_per_chunk;
+    tt = i - s * p.tiles_per_chunk;
+    j = (it.r - s + p.n_chunks) % p.n_chunks;
+  }
+  kv0 = j * p.chunk_len + tt * kBN;
+  kv_end = min(j * p.chunk_len + p.chunk_len, p.L);
+}
+
+// Wait used only while winding down: ignores the abort flag, keeps its own time limit.
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > ctl.limit_ns) {
+      if (ctl.status) atomicCAS(ctl.status, 0, kErrTimeout | (kSiteDrain << 8));
+      return;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    ring_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  static_assert(D == 64 || D == 128, "head dim");
+  constexpr int kBoxes = D / 64;                 // 64-column (128-byte) TMA boxes per row
+  constexpr uint32_t kBoxBytes = 128 * 64 * 2;   // 16 KB
+  constexpr uint32_t kTileBytes = kBoxes * kBoxBytes;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_smem = smem;                                  // 2 tiles
+  uint8_t* kv_smem = smem + 2 * kTileBytes;                // kStages tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kv_smem + kStages * kTileBytes);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;                  // [kStages]
+  uint64_t* kv_empty = bars + 1 + kStages;       // [kStages]
+  uint64_t* s_full = bars + 1 + 2 * kStages;     // [2]
+  uint64_t* p_full = bars + 3 + 2 * kStages;     // [2]
+  uint64_t* o_full = bars + 5 + 2 * kStages;
+  uint64_t* drain_bar = bars + 6 + 2 * kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * kStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* skip_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(&p_full[0], 4);
+    mbar_init(&p_full[1], 4);
+    mbar_init(o_full, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    // A launch whose status word already holds an error does no work: after one expired
+    // wait the remaining CTAs end at once instead of each running into its own limit.
+    *skip_flag = (p.status != nullptr && *reinterpret_cast<volatile int*>(p.status) != 0) ? 1 : 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (*skip_flag) return;  // uniform across the CTA (read after the barrier)
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const Item it = decode_item(p);
+
+  if (warp == kLoadWarp) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const uint64_t pol_kv = policy_evict_last();
+      const uint64_t pol_q = policy_evict_first();
+      const bool load_q = (p.debug_fault != 1);
+      if (load_q) {
+        mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
+#pragma unroll
+        for (int x = 0; x < kBoxes; ++x) {
+          tma_load_4d(q_smem + x * kBoxBytes, &tm_q, q_full, x * 64, it.rowA, it.headA, it.b, pol_q);
+          tma_load_4d(q_smem + kTileBytes + x * kBoxBytes, &tm_q, q_full, x * 64, it.rowB, it.headB, it.b, pol_q);
+        }
+      }
+      int slot = 0;
+      bool ok = true;
+      for (int i = 0; i < it.n_tiles && ok; ++i) {
+        int kv0, kv_end;
+        kv_tile(p, it, i, kv0, kv_end);
+#pragma unroll
+        for (int which = 0; which < 2; ++which, ++slot) {
+          const int st = slot % kStages;
+          const uint32_t ph = (slot / kStages) & 1;
+          if (!wait_bounded(&kv_empty[st], ph ^ 1, ctl, kSiteLoadEmpty)) { ok = false; break; }
+          mbar_arrive_expect_tx(&kv_full[st], kTileBytes);
+          const CUtensorMap* tm = which == 0 ? &tm_k : &tm_v;
+          uint8_t* dst = kv_smem + st * kTileBytes;
+#pragma unroll
+          for (int x = 0; x < kBoxes; ++x)
+            tma_load_4d(dst + x * kBoxBytes, tm, &kv_full[st], x * 64, kv0, it.g, it.b, pol_kv);
+        }
+      }
+      // drain: every load this thread issued has landed before the CTA can exit
+      if (load_q) wait_drain(q_full, 0, ctl);
+      for (int s2 = (slot > kStages ? slot - kStages : 0); s2 < slot; ++s2)
+        wait_drain(&kv_full[s2 % kStages], (s2 / kStages) & 1, ctl);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, kBN, false);
+      constexpr uint32_t idesc_o = make_idesc_bf16(128, D, true);
+      const uint32_t q_addr0 = smem_u32(q_smem);
+      const uint32_t kv_addr0 = smem_u32(kv_smem);
+
+      // S_ab = Q_ab K^T: M=128, N=128, K=D in steps of 16 (32 bytes inside a 128-byte swizzled row)
+      auto issue_s = [=](int ab, int st) {
+        const uint32_t kaddr = kv_addr0 + st * kTileBytes;
+        const uint32_t qaddr = q_addr0 + ab * kTileBytes;
+        const uint32_t d_tmem = tmem_base + ab * 256;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          umma_ss(d_tmem, make_sdesc(qaddr + off, 16, 1024), make_sdesc(kaddr + off, 16, 1024), idesc_s,
+                  kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_ab += P_ab V: A = P from TMEM (8 columns per 16 keys), B = V N-major (d contiguous)
+      auto issue_pv = [=](int ab, int st, bool acc) {
+        const uint32_t vaddr = kv_addr0 + st * kTileBytes;
+        const uint32_t p_tmem = tmem_base + ab * 256;
+        const uint32_t o_tmem = tmem_base + 128 + ab * 256;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          umma_ts(o_tmem, p_tmem + kk * 8, make_sdesc(vaddr + kk * 2048, kBoxBytes, 1024), idesc_o,
+                  (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = wait_bounded(q_full, 0, ctl, kSiteMmaQ);
+      tc_fence_after();
+      const int T = it.n_tiles;
+      int vst_prev = 0;
+      for (int i = 0; i < T && ok; ++i) {
+        const int kslot = 2 * i, vslot = 2 * i + 1;
+        const int kst = kslot % kStages, vst = vslot % kStages;
+        if (!wait_bounded(&kv_full[kst], (kslot / kStages) & 1, ctl, kSiteMmaKV)) { ok = false; break; }
+        tc_fence_after();
+        issue_s(0, kst);
+        umma_commit(&s_full[0]);
+        if (i > 0) {
+          if (!wait_bounded(&p_full[1], (i - 1) & 1, ctl, kSiteMmaP)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(1, vst_prev, i - 1 > 0);
+          umma_commit(&kv_empty[vst_prev]);
+        }
+        issue_s(1, kst);
+        umma_commit(&s_full[1]);
+        umma_commit(&kv_empty[kst]);
+        if (!wait_bounded(&kv_full[vst], (vslot / kStages) & 1, ctl, kSiteMmaKV)) { ok = false; break; }
+        if (!wait_bounded(&p_full[0], i & 1, ctl, kSiteMmaP)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(0, vst, i > 0);
+        vst_prev = vst;
+      }
+      if (ok && T > 0) {
+        if (wait_bounded(&p_full[1], (T - 1) & 1, ctl, kSiteMmaP)) {
+          tc_fence_after();
+          issue_pv(1, vst_prev, T - 1 > 0);
+          umma_commit(&kv_empty[vst_prev]);
+          umma_commit(o_full);
+        }
+      }
+      // drain: all MMAs issued by this thread are complete before TMEM is freed
+      umma_commit(drain_bar);
+      wait_drain(drain_bar, 0, ctl);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- softmax / correction / epilogue (warps 0-7) ----------------
+    const int ab = warp >> 2;                       // 0: tile A, 1: tile B
+    const uint32_t lane_base = (warp & 3) * 32;     // TMEM lane window of this warp
+    const int row_in_tile = lane_base + lane;
+    const int q_row = (ab == 0 ? it.rowA : it.rowB) + row_in_tile;
+    const int head = ab == 0 ? it.headA : it.headB;
+    const uint32_t tS = tmem_base + (ab ? 256u : 0u) + (lane_base << 16);
+    const uint32_t tO = tmem_base + (ab ? 384u : 128u) + (lane_base << 16);
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY;  // running max of scaled scores, log2 units
+    float l_run = 0.f;        // running sum of 2^(s*sl2 - m_run)
+    bool ok = true;
+
+    for (int i = 0; i < it.n_tiles; ++i) {
+      // warp-uniform decision: the TMEM loads below are .sync.aligned
+      if (!__all_sync(0xffffffffu, wait_bounded(&s_full[ab], i & 1, ctl, kSiteSoftS))) { ok = false; break; }
+      tc_fence_after();
+      int kv0, kv_end;
+      kv_tile(p, it, i, kv0, kv_end);
+      int lim = kv_end - kv0;
+      if (p.causal) lim = min(lim, q_row - kv0 + 1);
+
+      float s[kBN];
+#pragma unroll
+      for (int cc = 0; cc < kBN / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tS + cc * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[cc * 32 + e] = __uint_as_float(r[e]);
+      }
+      if (lim < kBN) {
+#pragma unroll
+        for (int e = 0; e < kBN; ++e)
+          if (e >= lim) s[e] = -INFINITY;
+      }
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+      for (int e = 4; e < kBN; e += 4) {
+        mx0 = fmaxf(mx0, s[e]);
+        mx1 = fmaxf(mx1, s[e + 1]);
+        mx2 = fmaxf(mx2, s[e + 2]);
+        mx3 = fmaxf(mx3, s[e + 3]);
+      }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      float alpha = 1.f;
+      if (m_tile > m_run + kRescaleThreshold) {
+        alpha = ex2_approx(m_run - m_tile);  // 0 when m_run = -inf
+        m_run = m_tile;
+        l_run *= alpha;
+      }
+      const float m_off = (m_run == -INFINITY) ? 0.f : m_run;
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < kBN / 32; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2_approx(fmaf(s[cc * 32 + 2 * e], sl2, -m_off));
+          const float p1 = ex2_approx(fmaf(s[cc * 32 + 2 * e + 1], sl2, -m_off));
+          sum0 += p0;
+          sum1 += p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + cc * 16, pk);
+      }
+      l_run += sum0 + sum1;
+      // O <- alpha * O for rows whose reference max moved (O holds the previous tiles' sum;
+      // PV of the previous tile has completed because S of this tile was issued after it).
+      if (i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(tO + cc * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(tO + cc * 32, r);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[ab]);
+    }
+
+    // ---------------- epilogue: O / l, LSE ----------------
+    if (ok && it.n_tiles > 0 && __all_sync(0xffffffffu, wait_bounded(o_full, 0, ctl, kSiteSoftO))) {
+      tc_fence_after();
+      const bool valid = (q_row < it.q_end) && (ab == 0 || p.pair_heads || it.rowB < it.q_end);
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      const long long orow = static_cast<long long>(q_row - p.out_row_base);
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tO + cc * 32, r);
+        tmem_wait_ld();
+        if (valid) {
+          if (p.out_fp32) {
+            float* dst = reinterpret_cast<float*>(p.o) + it.b * p.o_sb + head * p.o_sh + orow * p.o_sl + cc * 32;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              float4 v4 = make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
+                                      __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+              *reinterpret_cast<float4*>(dst + e) = v4;
+            }
+          } else {
+            __nv_bfloat16* dst =
+                reinterpret_cast<__nv_bfloat16*>(p.o) + it.b * p.o_sb + head * p.o_sh + orow * p.o_sl + cc * 32;
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 v4;
+              v4.x = pack_bf16x2(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
+              v4.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+              v4.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
+              v4.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
+              *reinterpret_cast<uint4*>(dst + e) = v4;
+            }
+          }
+        }
+      }
+      if (valid) {
+        const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+        p.lse[it.b * p.l_sb + head * p.l_sh + orow * p.l_sl] = lse;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// Dynamic shared memory: 1 KB alignment slack + Q (2 tiles) + KV ring + barriers.
+__host__ __device__ constexpr size_t fwd_smem_bytes(int d) {
+  return 1024 + static_cast<size_t>(2 + kStages) * 128 * d * 2 + 256;
+}
+
+}  // namespace cpattn

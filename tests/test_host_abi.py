@@ -1,0 +1,97 @@
+"""Host-side tests of the C ABI (no GPU): the library loads, exports every declared symbol,
+and plan validation / ring map / FLOP counts behave as the header states."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sequence_long_context_ring_b200 import binding, build
+from sequence_long_context_ring_b200.binding import Plan, CpError
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(cp_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = binding.lib()
+    declared = _declared_functions()
+    assert "cp_attn_fwd" in declared and "cp_layout_seq2head" in declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(binding.EXPORTS) <= set(declared)
+
+
+def test_version_and_status_strings():
+    lib = binding.lib()
+    assert b"sm_100a" in lib.cp_version()
+    for st in range(-6, 1):
+        assert lib.cp_status_string(st)
+
+
+@pytest.mark.parametrize("kw,err", [
+    (dict(Hq=6, Hkv=4), binding.CP_ERR_INVALID_ARG),            # Hq % Hkv != 0
+    (dict(L=1000, n_cp=3), binding.CP_ERR_INVALID_ARG),         # L % N != 0
+    (dict(d=96), binding.CP_ERR_UNSUPPORTED),                    # d not in {64, 128}
+    (dict(n_hp=2), binding.CP_ERR_INVALID_ARG),                  # ring needs n_hp == 1
+    (dict(mode="ulysses", n_cp=3, L=999), binding.CP_ERR_INVALID_ARG),   # H % N != 0
+    (dict(mode="ulysses", Hq=32, Hkv=4, n_cp=8), binding.CP_ERR_INVALID_ARG),  # degree > KV groups
+    (dict(mode="2d", n_hp=3, n_cp=2), binding.CP_ERR_INVALID_ARG),       # Hq % n_hp != 0
+    (dict(split="zigzag"), binding.CP_ERR_UNSUPPORTED),
+    (dict(B=0), binding.CP_ERR_INVALID_ARG),
+])
+def test_plan_validation_errors(kw, err):
+    args = dict(B=1, Hq=8, Hkv=8, L=1024, d=128, n_cp=4)
+    args.update(kw)
+    with pytest.raises(CpError) as e:
+        Plan(**args)
+    assert e.value.status == err
+
+
+def test_ring_map_and_skip_set():
+    # step s: rank r holds chunk (r - s) mod N; j > r skipped, j == r diagonal.
+    p = Plan(B=1, Hq=4, Hkv=4, L=1024, d=64, n_cp=4)
+    for r in range(4):
+        seen = []
+        for s in range(4):
+            j, kind = p.step_chunk(r, s)
+            assert j == (r - s) % 4
+            assert kind == (0 if j > r else 2 if j == r else 1)
+            seen.append(j)
+        assert sorted(seen) == [0, 1, 2, 3]
+    with pytest.raises(CpError):
+        p.step_chunk(4, 0)
+    nc = Plan(B=1, Hq=4, Hkv=4, L=1024, d=64, n_cp=4, causal=False)
+    assert all(nc.step_chunk(r, s)[1] == 1 for r in range(4) for s in range(4))
+
+
+def test_flops_and_work_items():
+    p = Plan(B=1, Hq=32, Hkv=8, L=212992, d=128, n_cp=16)
+    assert abs(p.flops() - 4 * 32 * 128 * 212992 * 212993 / 2) < 1.0
+    assert abs(p.flops(True) - 2.5 * p.flops()) < 1.0
+    # GQA pairs two heads of a group at the same 128 query rows: 8 KV heads x 2 pairs x 1664 tiles
+    assert p.num_work_items() == 8 * 2 * 16 * 104
+    m = Plan(B=1, Hq=4, Hkv=4, L=1024, d=64, n_cp=4)
+    assert m.num_work_items() == 4 * 4 * 1  # MHA: two consecutive tiles of a 256-row chunk
+
+
+def test_workspace_sizes():
+    p = Plan(B=1, Hq=32, Hkv=32, L=131072, d=128, n_cp=8, mode="ulysses")
+    assert p.workspace_size(False) >= 4 * 32 * 131072 * 128 * 2
+    r = Plan(B=1, Hq=4, Hkv=4, L=1024, d=64, n_cp=4)
+    assert r.workspace_size(False) == 0
+    assert r.workspace_size(True) >= 4 * 1024 * 64 * 4
