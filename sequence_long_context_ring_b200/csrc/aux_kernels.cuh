@@ -144,10 +144,11 @@ __global__ void __launch_bounds__(256) rowdot_kernel(const DotParams p) {
   if (live && vec == 0) p.D[b * p.D_sb + h * p.D_sh + l * p.D_sl] = acc;
 }
 
-// ---- dQ accumulator (fp32, already scaled) -> bf16 output ------------------------------------
+// ---- dQ accumulator (fp32) * scale -> bf16 output ------------------------------------
 struct CastParams {
   const float* src;      // contiguous [B, H, L, d]
   __nv_bfloat16* dst;
+  float scale;           // applied before rounding
   int B, H, L, d;
   long long d_sb, d_sh, d_sl;
 };
@@ -164,8 +165,8 @@ __global__ void __launch_bounds__(256) cast_bf16_kernel(const CastParams p) {
   const int h = static_cast<int>(t % p.H);
   const int b = static_cast<int>(t / p.H);
   const float4 v = reinterpret_cast<const float4*>(p.src)[i];
-  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x * p.scale, v.y * p.scale);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(v.z * p.scale, v.w * p.scale);
   uint2 packed;
   packed.x = *reinterpret_cast<uint32_t*>(&lo);
   packed.y = *reinterpret_cast<uint32_t*>(&hi);

@@ -1,11 +1,461 @@
-// bwd_kernel.cuh — backward of ring attention for sm_100a (recompute from the stored LSE).
+// bwd_kernel.cuh — ring-attention backward for sm_100a (tcgen05 + TMEM + TMA), recomputing
+// the probabilities from the forward's stored LSE instead of storing them ("スケーラビリティと
+// メモリ管理" in "長いシーケンスのLLMトレーニングの進展": keep only what is needed, recompute
+// the rest).  Gradients of O = softmax(scale Q K^T) V, per KV head g and query head h of its
+// group:  P = exp(scale S - LSE);  dV += P^T dO;  dP = dO V^T;  dS = P o (dP - D) with
+// D = rowsum(dO o O);  dQ += scale dS K;  dK += scale dS^T Q.
+//
+// Ring order: the CTA owns one 128-row KV tile of chunk j and visits the query chunks of the
+// ranks that see it — r = j (the diagonal chunk, masked key <= query), j+1, ..., N-1 — and,
+// for each 128-row query tile, every query head of the KV group.  dK and dV accumulate in
+// TMEM over the whole visit (the sum over the group's heads happens there, without atomics);
+// dQ is added into an fp32 accumulator in global memory.
+//
+// Warp roles (320 threads):
+//   warps 0-3  P / dS warps: thread t <-> key row t <-> TMEM lane t; epilogue writes dK, dV
+//   warps 4-7  dQ warps: thread t <-> query row t of the dQ tile; float4 atomics into dQ_acc
+//   warp  8    loads: K, V once (TMA); per query tile Q_i, dO_i (TMA, 2 stages) and
+//              LSE_i, D_i (plain loads into shared memory)
+//   warp  9    MMA issuer (one thread)
+// TMEM columns: S^T/P^T [0,128)  dP^T/dS^T, then dQ [128,256)  dV [256,384)  dK [384,512).
 #pragma once
 #include <cstddef>
 #include "sm100.cuh"
 
 namespace cpattn {
 
+constexpr int kBwdThreads = 320;
+constexpr uint32_t kBwdTmemCols = 512;
+
 // Extra workspace the backward kernels need beyond the dQ accumulator and D.
 inline size_t bwd_workspace_extra(int, int, int, int, int) { return 0; }
+
+enum BwdSite : int {
+  kBSiteLoadEmpty = 17, kBSiteMmaKV = 18, kBSiteMmaQ = 19, kBSiteMmaDq = 20, kBSiteMmaP = 21,
+  kBSiteMmaDs = 22, kBSiteSoftS = 23, kBSiteSoftDp = 24, kBSiteDqFull = 25, kBSiteDone = 26,
+};
+
+struct BwdParams {
+  int B, Hq, Hkv, L, d, G;
+  int n_chunks, chunk_len, tiles_per_chunk;
+  int causal;
+  float scale;        // softmax scale (dQ, dK factor)
+  float scale_log2;   // scale * log2(e)
+  const float* lse;   // [B, Hq, L] natural-log LSE of the forward
+  long long lse_sb, lse_sh, lse_sl;
+  const float* Dvec;  // [B, Hq, L] rowsum(dO * O), contiguous
+  float* dq_acc;      // [B, Hq, L, d] fp32, contiguous, zeroed before the launch
+  __nv_bfloat16* dk;  // [B, Hkv, L, d]
+  long long dk_sb, dk_sh, dk_sl;
+  __nv_bfloat16* dv;
+  long long dv_sb, dv_sh, dv_sl;
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+
+struct BwdItem {
+  int b, g, j, kv0, kv_end;  // KV tile rows [kv0, min(kv0+128, kv_end))
+  int first_qtile;           // first query tile (in chunk j) that sees the KV tile
+  int n_qtiles;              // query tiles visited (each for all G heads)
+  int n_iter;                // n_qtiles * G
+};
+
+__device__ __forceinline__ BwdItem decode_bwd_item(const BwdParams& p) {
+  BwdItem it;
+  const int n_inner = p.B * p.Hkv;
+  const int pos = blockIdx.x / n_inner;        // longest first: the earliest keys see the most queries
+  const int inner = blockIdx.x - pos * n_inner;
+  it.b = inner / p.Hkv;
+  it.g = inner - it.b * p.Hkv;
+  it.j = pos / p.tiles_per_chunk;
+  const int tt = pos - it.j * p.tiles_per_chunk;
+  const int c0 = it.j * p.chunk_len;
+  it.kv0 = c0 + tt * 128;
+  it.kv_end = min(c0 + p.chunk_len, p.L);
+  if (p.causal) {
+    it.first_qtile = tt;  // query tiles are aligned to the chunk start like the KV tiles
+    it.n_qtiles = (p.tiles_per_chunk - tt) + (p.n_chunks - 1 - it.j) * p.tiles_per_chunk;
+  } else {
+    it.first_qtile = 0;
+    it.n_qtiles = p.n_chunks * p.tiles_per_chunk;
+  }
+  it.n_iter = it.n_qtiles * p.G;
+  return it;
+}
+
+// i-th iteration -> query head and first row of the query tile, and the end of its chunk.
+__device__ __forceinline__ void bwd_qtile(const BwdParams& p, const BwdItem& it, int i, int& h, int& q0,
+                                          int& q_end) {
+  const int t = i / p.G;
+  h = it.g * p.G + (i - t * p.G);
+  int r, tq;
+  if (p.causal) {
+    const int first_len = p.tiles_per_chunk - it.first_qtile;
+    if (t < first_len) {
+      r = it.j;
+      tq = it.first_qtile + t;
+    } else {
+      const int t2 = t - first_len;
+      const int qq = t2 / p.tiles_per_chunk;
+      r = it.j + 1 + qq;
+      tq = t2 - qq * p.tiles_per_chunk;
+    }
+  } else {
+    // ring order starting at the diagonal chunk: r = j, j+1, ... (mod N)
+    const int s = t / p.tiles_per_chunk;
+    tq = t - s * p.tiles_per_chunk;
+    r = (it.j + s) % p.n_chunks;
+  }
+  q0 = r * p.chunk_len + tq * 128;
+  q_end = min(r * p.chunk_len + p.chunk_len, p.L);
+}
+
+__device__ __forceinline__ void bwd_wait_drain(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > ctl.limit_ns) {
+      if (ctl.status) atomicCAS(ctl.status, 0, kErrTimeout | (kBSiteDone << 8));
+      return;
+    }
+  }
+}
+
+// Shared memory (d = 128): K 32K | V 32K | Q[2] 64K | dO[2] 64K | dS 32K | LSE/D[2] 2K | barriers.
+// The dS tile is 128 keys x 128 queries whatever d is.
+constexpr size_t kBwdDsBytes = 128 * 128 * 2;
+__host__ __device__ constexpr size_t bwd_smem_bytes(int d) {
+  return static_cast<size_t>(6) * 128 * d * 2 + kBwdDsBytes + 2 * 1024 + 256;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    ring_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  constexpr int kBoxes = D / 64;
+  constexpr uint32_t kBoxBytes = 128 * 64 * 2;
+  constexpr uint32_t kTile = kBoxes * kBoxBytes;  // one 128-row bf16 tile
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* k_s = smem;
+  uint8_t* v_s = smem + kTile;
+  uint8_t* q_s = smem + 2 * kTile;    // [2]
+  uint8_t* do_s = smem + 4 * kTile;   // [2]
+  uint8_t* ds_s = smem + 6 * kTile;   // dS, query-major halves of 64 queries (16 KB each)
+  float* stat_s = reinterpret_cast<float*>(smem + 6 * kTile + kBwdDsBytes);  // [2][256]: lse2, D
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * kTile + kBwdDsBytes + 2048);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;     // [2]
+  uint64_t* q_empty = bars + 3;    // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* dp_full = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* ds_full = bars + 8;
+  uint64_t* dq_full = bars + 9;
+  uint64_t* dq_free = bars + 10;
+  uint64_t* done_bar = bars + 11;
+  uint64_t* drain_bar = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* skip_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(ds_full, 4);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 4);
+    mbar_init(done_bar, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    // the shared-memory layout needs a 1 KB aligned base for the 128-byte swizzle atoms
+    const bool misaligned = (smem_u32(smem) & 1023u) != 0;
+    const bool poisoned = p.status != nullptr && *reinterpret_cast<volatile int*>(p.status) != 0;
+    if (misaligned && p.status) atomicCAS(p.status, 0, 3 /* alignment */ | (31 << 8));
+    *skip_flag = (misaligned || poisoned) ? 1 : 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (*skip_flag) return;
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kBwdTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const BwdItem it = decode_bwd_item(p);
+  const uint32_t tS = tmem_base, tDP = tmem_base + 128, tDV = tmem_base + 256, tDK = tmem_base + 384;
+
+  if (warp == 8) {
+    // ---------------- loads ----------------
+    const uint64_t pol_keep = policy_evict_last();
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(kv_full, 2 * kTile);
+#pragma unroll
+      for (int x = 0; x < kBoxes; ++x) {
+        tma_load_4d(k_s + x * kBoxBytes, &tm_k, kv_full, x * 64, it.kv0, it.g, it.b, pol_keep);
+        tma_load_4d(v_s + x * kBoxBytes, &tm_v, kv_full, x * 64, it.kv0, it.g, it.b, pol_keep);
+      }
+    }
+    bool ok = true;
+    int issued = 0;
+    for (int i = 0; i < it.n_iter && ok; ++i) {
+      const int st = i & 1;
+      const uint32_t ph = (i >> 1) & 1;
+      ok = __all_sync(0xffffffffu, wait_bounded(&q_empty[st], ph ^ 1, ctl, kBSiteLoadEmpty));
+      if (!ok) break;
+      int h, q0, q_end;
+      bwd_qtile(p, it, i, h, q0, q_end);
+      // LSE (log2 units) and D of the tile's 128 query rows; rows outside the chunk get
+      // LSE = +inf (probability 0) so they contribute nothing.
+      float* lse2 = stat_s + st * 256;
+      float* dvec = lse2 + 128;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int rr = lane * 4 + u;
+        const int q = q0 + rr;
+        float l2 = INFINITY, dd = 0.f;
+        if (q < q_end) {
+          l2 = p.lse[it.b * p.lse_sb + h * p.lse_sh + static_cast<long long>(q) * p.lse_sl] *
+               1.4426950408889634f;
+          dd = p.Dvec[(static_cast<long long>(it.b) * p.Hq + h) * p.L + q];
+        }
+        lse2[rr] = l2;
+        dvec[rr] = dd;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&q_full[st], 2 * kTile);  // the arrive also publishes lse2 / D
+#pragma unroll
+        for (int x = 0; x < kBoxes; ++x) {
+          tma_load_4d(q_s + st * kTile + x * kBoxBytes, &tm_q, &q_full[st], x * 64, q0, h, it.b, pol_keep);
+          tma_load_4d(do_s + st * kTile + x * kBoxBytes, &tm_do, &q_full[st], x * 64, q0, h, it.b, pol_keep);
+        }
+      }
+      ++issued;
+    }
+    if (lane == 0) {
+      bwd_wait_drain(kv_full, 0, ctl);
+      for (int s2 = (issued > 2 ? issued - 2 : 0); s2 < issued; ++s2) bwd_wait_drain(&q_full[s2 & 1], (s2 >> 1) & 1, ctl);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_kk = make_idesc_bf16(128, 128, false);     // S^T, dP^T: both K-major
+      constexpr uint32_t idesc_tn = make_idesc_bf16(128, D, true);        // dV, dK: A TMEM, B N-major
+      constexpr uint32_t idesc_nn = make_idesc_bf16(128, D, true) | (1u << 15);  // dQ: A, B N-major
+      const uint32_t k_a = smem_u32(k_s), v_a = smem_u32(v_s), ds_a = smem_u32(ds_s);
+      bool ok = wait_bounded(kv_full, 0, ctl, kBSiteMmaKV);
+      for (int i = 0; i < it.n_iter && ok; ++i) {
+        const int st = i & 1;
+        const uint32_t q_a = smem_u32(q_s + st * kTile), do_a = smem_u32(do_s + st * kTile);
+        if (!wait_bounded(&q_full[st], (i >> 1) & 1, ctl, kBSiteMmaQ)) { ok = false; break; }
+        tc_fence_after();
+        // (1) S^T = K Q^T  [M = keys, N = queries, K = d]
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          umma_ss(tS, make_sdesc(k_a + off, 16, 1024), make_sdesc(q_a + off, 16, 1024), idesc_kk, kk > 0);
+        }
+        umma_commit(s_full);
+        // (2) dP^T = V dO^T, into the columns that held dQ of the previous tile
+        if (i > 0 && !wait_bounded(dq_free, (i - 1) & 1, ctl, kBSiteMmaDq)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          umma_ss(tDP, make_sdesc(v_a + off, 16, 1024), make_sdesc(do_a + off, 16, 1024), idesc_kk, kk > 0);
+        }
+        umma_commit(dp_full);
+        // (3) dV += P^T dO  [A = P^T in TMEM (keys x queries), B = dO N-major]
+        if (!wait_bounded(p_full, i & 1, ctl, kBSiteMmaP)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ts(tDV, tS + kk * 8, make_sdesc(do_a + kk * 2048, kBoxBytes, 1024), idesc_tn, (i > 0 || kk > 0));
+        // (4) dK += dS^T Q  [A = dS^T in TMEM, B = Q N-major]
+        if (!wait_bounded(ds_full, i & 1, ctl, kBSiteMmaDs)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ts(tDK, tDP + kk * 8, make_sdesc(q_a + kk * 2048, kBoxBytes, 1024), idesc_tn, (i > 0 || kk > 0));
+        // (5) dQ_i = dS K  [A = dS query-major in smem, B = K N-major], over dP^T/dS^T
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ss(tDP, make_sdesc(ds_a + kk * 2048, kBoxBytes, 1024), make_sdesc(k_a + kk * 2048, kBoxBytes, 1024),
+                  idesc_nn, kk > 0);
+        umma_commit(dq_full);
+        umma_commit(&q_empty[st]);
+      }
+      if (ok) umma_commit(done_bar);
+      umma_commit(drain_bar);
+      bwd_wait_drain(drain_bar, 0, ctl);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ---------------- P / dS (thread = key row) and the dK / dV epilogue ----------------
+    const uint32_t lane_base = warp * 32;
+    const int t = lane_base + lane;
+    const int kv_row = it.kv0 + t;
+    const bool kv_live = kv_row < it.kv_end;
+    const uint32_t lofs = lane_base << 16;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int i = 0; i < it.n_iter; ++i) {
+      const int st = i & 1;
+      int h, q0, q_end;
+      bwd_qtile(p, it, i, h, q0, q_end);
+      const float* lse2 = stat_s + st * 256;
+      const float* dvec = lse2 + 128;
+      // causal: query columns c < kv_row - q0 do not see this key
+      const int c_lo = p.causal ? (kv_row - q0) : 0;
+      if (!__all_sync(0xffffffffu, wait_bounded(s_full, i & 1, ctl, kBSiteSoftS))) { ok = false; break; }
+      tc_fence_after();
+      uint32_t pk[64];  // P^T row as bf16 pairs, kept for dS
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tS + lofs + cc * 32, r);
+        tmem_wait_ld();
+        uint32_t pst[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int c = cc * 32 + e;
+          float p0 = ex2_approx(fmaf(__uint_as_float(r[e]), sl2, -lse2[c]));
+          float p1 = ex2_approx(fmaf(__uint_as_float(r[e + 1]), sl2, -lse2[c + 1]));
+          if (!kv_live || c < c_lo) p0 = 0.f;
+          if (!kv_live || c + 1 < c_lo) p1 = 0.f;
+          pst[e >> 1] = pack_bf16x2(p0, p1);
+          pk[c >> 1] = pst[e >> 1];
+        }
+        // P^T columns [16cc, 16cc+16) overwrite S^T columns already read (in-place stream)
+        tmem_st16(tS + lofs + cc * 16, pst);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+
+      if (!__all_sync(0xffffffffu, wait_bounded(dp_full, i & 1, ctl, kBSiteSoftDp))) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tDP + lofs + cc * 32, r);
+        tmem_wait_ld();
+        uint32_t dsk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int c = cc * 32 + e;
+          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[c >> 1]));
+          const float d0 = pp.x * (__uint_as_float(r[e]) - dvec[c]);
+          const float d1 = pp.y * (__uint_as_float(r[e + 1]) - dvec[c + 1]);
+          dsk[e >> 1] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tDP + lofs + cc * 16, dsk);
+        // dS for the dQ MMA: query-major, two 64-query halves of [128 keys x 128 B], 128-byte
+        // swizzle (16-byte chunk index XOR key row % 8); this chunk = queries [32cc, 32cc+32)
+        uint8_t* half = ds_s + (cc >> 1) * kBoxBytes + t * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int chunk = (cc & 1) * 4 + u;
+          *reinterpret_cast<uint4*>(half + ((chunk ^ (t & 7)) << 4)) =
+              make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]);
+        }
+      }
+      tmem_wait_st();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
+    }
+    // epilogue: dV, dK (scaled) for this thread's key row
+    const bool have = it.n_iter > 0;
+    if (ok && (!have || __all_sync(0xffffffffu, wait_bounded(done_bar, 0, ctl, kBSiteDone)))) {
+      tc_fence_after();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tsrc = (which == 0 ? tDV : tDK) + lofs;
+        const float f = which == 0 ? 1.f : p.scale;
+        __nv_bfloat16* dst = which == 0 ? p.dv + it.b * p.dv_sb + it.g * p.dv_sh + static_cast<long long>(kv_row) * p.dv_sl
+                                        : p.dk + it.b * p.dk_sb + it.g * p.dk_sh + static_cast<long long>(kv_row) * p.dk_sl;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          if (have) {
+            tmem_ld32(tsrc + cc * 32, r);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;
+          }
+          if (kv_live) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 v4;
+              v4.x = pack_bf16x2(__uint_as_float(r[e]) * f, __uint_as_float(r[e + 1]) * f);
+              v4.y = pack_bf16x2(__uint_as_float(r[e + 2]) * f, __uint_as_float(r[e + 3]) * f);
+              v4.z = pack_bf16x2(__uint_as_float(r[e + 4]) * f, __uint_as_float(r[e + 5]) * f);
+              v4.w = pack_bf16x2(__uint_as_float(r[e + 6]) * f, __uint_as_float(r[e + 7]) * f);
+              *reinterpret_cast<uint4*>(dst + cc * 32 + e) = v4;
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // ---------------- dQ (warps 4-7, thread = query row of the tile) ----------------
+    const uint32_t lane_base = (warp & 3) * 32;
+    const int t = lane_base + lane;
+    const uint32_t lofs = lane_base << 16;
+    for (int i = 0; i < it.n_iter; ++i) {
+      int h, q0, q_end;
+      bwd_qtile(p, it, i, h, q0, q_end);
+      const int q = q0 + t;
+      if (!__all_sync(0xffffffffu, wait_bounded(dq_full, i & 1, ctl, kBSiteDqFull))) break;
+      tc_fence_after();
+      float* dst = p.dq_acc + ((static_cast<long long>(it.b) * p.Hq + h) * p.L + q) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tDP + lofs + cc * 32, r);
+        tmem_wait_ld();
+        if (q < q_end) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            atomicAdd(reinterpret_cast<float4*>(dst + cc * 32 + e),
+                      make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                                  __uint_as_float(r[e + 3])));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kBwdTmemCols);
+  }
+}
 
 }  // namespace cpattn

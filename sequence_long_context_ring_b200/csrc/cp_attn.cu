@@ -241,13 +241,178 @@ cp_status_t head_buf_to_seq(const void* buf, cp_tensor_t* out, cudaStream_t s) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+template <int D>
+cp_status_t launch_bwd_d(const BwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const CUtensorMap& mdo, int64_t grid, cudaStream_t s) {
+  const size_t smem = bwd_smem_bytes(D);
+  if (cudaFuncSetAttribute(ring_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return CP_ERR_CUDA;
+  ring_bwd_kernel<D><<<(unsigned)grid, kBwdThreads, smem, s>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+// D = rowsum(dO * O) for [b, h, l] rows given by per-axis element strides.
+cp_status_t launch_rowdot(const void* o, const int64_t os[3], const void* g, const int64_t gs[3], float* D, int B,
+                          int H, int L, int d, cudaStream_t s) {
+  DotParams p{static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(g), D, B, H, L, d,
+              os[0], os[1], os[2], gs[0], gs[1], gs[2], (int64_t)H * L, (int64_t)L, 1};
+  const int64_t threads = (int64_t)B * H * L * (d / 8);
+  if (threads == 0) return CP_OK;
+  rowdot_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status_t launch_cast(const float* src, __nv_bfloat16* dst, float scale, int B, int H, int L, int d, int64_t sb,
+                        int64_t sh, int64_t sl, cudaStream_t s) {
+  CastParams p{src, dst, scale, B, H, L, d, sb, sh, sl};
+  const int64_t n4 = (int64_t)B * H * L * d / 4;
+  if (n4 == 0) return CP_OK;
+  cast_bf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
 cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_tensor_t* k, const cp_tensor_t* v,
                          const cp_tensor_t* o, const cp_tensor_t* lse, const cp_tensor_t* dout, cp_tensor_t* dq,
                          cp_tensor_t* dk, cp_tensor_t* dv, void* ws, size_t ws_bytes, void* stream) {
-  (void)q; (void)k; (void)v; (void)o; (void)lse; (void)dout; (void)dq; (void)dk; (void)dv;
-  (void)ws; (void)ws_bytes; (void)stream;
   if (!plan) return CP_ERR_INVALID_ARG;
-  return CP_ERR_UNSUPPORTED;
+  const cp_attn_config_t& c = plan->cfg;
+  const cudaStream_t s = as_stream(stream);
+  const bool seq = c.mode != CP_MODE_RING;
+  if (!seq) {
+    CP_TRY(check4(q, CP_BF16, c.B, c.Hq, c.L, c.d));
+    CP_TRY(check4(k, CP_BF16, c.B, c.Hkv, c.L, c.d));
+    CP_TRY(check4(v, CP_BF16, c.B, c.Hkv, c.L, c.d));
+    CP_TRY(check4(o, CP_BF16, c.B, c.Hq, c.L, c.d));
+    CP_TRY(check4(dout, CP_BF16, c.B, c.Hq, c.L, c.d));
+    CP_TRY(check4(dq, CP_BF16, c.B, c.Hq, c.L, c.d));
+    CP_TRY(check4(dk, CP_BF16, c.B, c.Hkv, c.L, c.d));
+    CP_TRY(check4(dv, CP_BF16, c.B, c.Hkv, c.L, c.d));
+  } else {
+    CP_TRY(check4(q, CP_BF16, c.B, c.L, c.Hq, c.d));
+    CP_TRY(check4(k, CP_BF16, c.B, c.L, c.Hkv, c.d));
+    CP_TRY(check4(v, CP_BF16, c.B, c.L, c.Hkv, c.d));
+    CP_TRY(check4(o, CP_BF16, c.B, c.L, c.Hq, c.d));
+    CP_TRY(check4(dout, CP_BF16, c.B, c.L, c.Hq, c.d));
+    CP_TRY(check4(dq, CP_BF16, c.B, c.L, c.Hq, c.d));
+    CP_TRY(check4(dk, CP_BF16, c.B, c.L, c.Hkv, c.d));
+    CP_TRY(check4(dv, CP_BF16, c.B, c.L, c.Hkv, c.d));
+  }
+  CP_TRY(check3(lse, c.B, c.Hq, c.L));
+  size_t need = 0;
+  cp_attn_workspace_size(plan, 1, &need);
+  if (!ws || ws_bytes < need) return CP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return CP_ERR_ALIGNMENT;
+  cp_status_t err = CP_OK;
+  int* sw = status_word(plan, &err);
+  if (!sw) return err;
+
+  const size_t nq = (size_t)c.B * c.Hq * c.L * c.d, nkv = (size_t)c.B * c.Hkv * c.L * c.d;
+  const size_t nrow = (size_t)c.B * c.Hq * c.L;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* dq_acc = reinterpret_cast<float*>(w);
+  w += align256(nq * 4);
+  float* Dvec = reinterpret_cast<float*>(w);
+  w += align256(nrow * 4);
+
+  // D = rowsum(dO * O): strides along (b, h, l) of o and dout in either layout
+  const int64_t os[3] = {o->stride[0], seq ? o->stride[2] : o->stride[1], seq ? o->stride[1] : o->stride[2]};
+  const int64_t gs[3] = {dout->stride[0], seq ? dout->stride[2] : dout->stride[1],
+                         seq ? dout->stride[1] : dout->stride[2]};
+  CP_TRY(launch_rowdot(o->data, os, dout->data, gs, Dvec, c.B, c.Hq, c.L, c.d, s));
+  if (cudaMemsetAsync(dq_acc, 0, nq * 4, s) != cudaSuccess) return CP_ERR_CUDA;
+
+  View vq, vk, vv, vdo;
+  void *dqh = nullptr, *dkh = nullptr, *dvh = nullptr;
+  if (!seq) {
+    vq = view_of(q);
+    vk = view_of(k);
+    vv = view_of(v);
+    vdo = view_of(dout);
+  } else {
+    void* qh = w;
+    w += align256(nq * 2);
+    void* doh = w;
+    w += align256(nq * 2);
+    dqh = w;
+    w += align256(nq * 2);
+    void* kh = w;
+    w += align256(nkv * 2);
+    void* vh = w;
+    w += align256(nkv * 2);
+    dkh = w;
+    w += align256(nkv * 2);
+    dvh = w;
+    // all-to-all seq -> head of the inputs and of the upstream gradient (the extra a2a of the
+    // backward, "05. 長系列の分散学習（Context Parallelism）" §3)
+    CP_TRY(seq_to_head_buf(q, qh, s));
+    CP_TRY(seq_to_head_buf(k, kh, s));
+    CP_TRY(seq_to_head_buf(v, vh, s));
+    CP_TRY(seq_to_head_buf(dout, doh, s));
+    vq = contiguous_view(qh, c.B, c.Hq, c.L, c.d);
+    vk = contiguous_view(kh, c.B, c.Hkv, c.L, c.d);
+    vv = contiguous_view(vh, c.B, c.Hkv, c.L, c.d);
+    vdo = contiguous_view(doh, c.B, c.Hq, c.L, c.d);
+  }
+
+  BwdParams p{};
+  p.B = c.B;
+  p.Hq = c.Hq;
+  p.Hkv = c.Hkv;
+  p.L = c.L;
+  p.d = c.d;
+  p.G = plan->G;
+  p.n_chunks = c.mode == CP_MODE_ULYSSES ? 1 : c.n_cp;
+  p.chunk_len = c.L / p.n_chunks;
+  p.tiles_per_chunk = (p.chunk_len + 127) / 128;
+  p.causal = c.causal ? 1 : 0;
+  p.scale = plan->scale;
+  p.scale_log2 = static_cast<float>(static_cast<double>(plan->scale) * 1.4426950408889634);
+  p.lse = static_cast<const float*>(lse->data);
+  p.lse_sb = lse->stride[0];
+  p.lse_sh = lse->stride[1];
+  p.lse_sl = lse->stride[2];
+  p.Dvec = Dvec;
+  p.dq_acc = dq_acc;
+  if (!seq) {
+    p.dk = static_cast<__nv_bfloat16*>(dk->data);
+    p.dk_sb = dk->stride[0];
+    p.dk_sh = dk->stride[1];
+    p.dk_sl = dk->stride[2];
+    p.dv = static_cast<__nv_bfloat16*>(dv->data);
+    p.dv_sb = dv->stride[0];
+    p.dv_sh = dv->stride[1];
+    p.dv_sl = dv->stride[2];
+  } else {
+    p.dk = static_cast<__nv_bfloat16*>(dkh);
+    p.dv = static_cast<__nv_bfloat16*>(dvh);
+    p.dk_sb = p.dv_sb = (int64_t)c.Hkv * c.L * c.d;
+    p.dk_sh = p.dv_sh = (int64_t)c.L * c.d;
+    p.dk_sl = p.dv_sl = c.d;
+  }
+  p.status = sw;
+  p.wait_limit_ns = c.wait_limit_ns ? c.wait_limit_ns : kDefaultWaitLimitNs;
+  CUtensorMap mq, mk, mv, mdo;
+  CP_TRY(make_map_bhld(&mq, vq.data, vq.B, vq.H, vq.L, vq.d, vq.sB, vq.sH, vq.sL));
+  CP_TRY(make_map_bhld(&mk, vk.data, vk.B, vk.H, vk.L, vk.d, vk.sB, vk.sH, vk.sL));
+  CP_TRY(make_map_bhld(&mv, vv.data, vv.B, vv.H, vv.L, vv.d, vv.sB, vv.sH, vv.sL));
+  CP_TRY(make_map_bhld(&mdo, vdo.data, vdo.B, vdo.H, vdo.L, vdo.d, vdo.sB, vdo.sH, vdo.sL));
+  const int64_t grid = (int64_t)p.n_chunks * p.tiles_per_chunk * c.B * c.Hkv;
+  if (c.d == 128) {
+    CP_TRY(launch_bwd_d<128>(p, mq, mk, mv, mdo, grid, s));
+  } else {
+    CP_TRY(launch_bwd_d<64>(p, mq, mk, mv, mdo, grid, s));
+  }
+  if (!seq) {
+    return launch_cast(dq_acc, static_cast<__nv_bfloat16*>(dq->data), plan->scale, c.B, c.Hq, c.L, c.d,
+                       dq->stride[0], dq->stride[1], dq->stride[2], s);
+  }
+  CP_TRY(launch_cast(dq_acc, static_cast<__nv_bfloat16*>(dqh), plan->scale, c.B, c.Hq, c.L, c.d,
+                     (int64_t)c.Hq * c.L * c.d, (int64_t)c.L * c.d, c.d, s));
+  // all-to-all head -> seq of the gradients
+  CP_TRY(head_buf_to_seq(dqh, dq, s));
+  CP_TRY(head_buf_to_seq(dkh, dk, s));
+  return head_buf_to_seq(dvh, dv, s);
 }
 
 }  // namespace
