@@ -29,10 +29,13 @@ def _probs(q, k, lse_row, rows, causal, scale):
     return np.exp(s - lse_row[:, None])
 
 
-def attention_backward(q, k, v, do, causal: bool = True, scale: float | None = None):
+def attention_backward(q, k, v, do, causal: bool = True, scale: float | None = None, o=None):
     """q [B,Hq,L,d], k/v [B,Hkv,L,d], do [B,Hq,L,d] (float64) -> dq, dk, dv (same shapes).
 
-    LSE and O are recomputed here from q, k, v (the plain definition)."""
+    P is recomputed here from q, k (the plain definition).  ``o`` is the forward output the
+    backward is given, used only in D = rowsum(dO * O): the backward works from the stored
+    forward state (recompute, do not store), and what the forward stores is its output as
+    written (bf16).  Default: the exact O."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
@@ -55,10 +58,10 @@ def attention_backward(q, k, v, do, causal: bool = True, scale: float | None = N
             m = s.max(axis=1)
             lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
             p = np.exp(s - lse[:, None])
-            o = p @ v[b, g]
+            o_bh = p @ v[b, g] if o is None else np.asarray(o[b, h], np.float64)
             dv[b, g] += p.T @ do[b, h]
             dp = do[b, h] @ v[b, g].T
-            D = (do[b, h] * o).sum(axis=1)
+            D = (do[b, h] * o_bh).sum(axis=1)
             ds = p * (dp - D[:, None])
             dq[b, h] = scale * (ds @ k[b, g])
             dk[b, g] += scale * (ds.T @ q[b, h])

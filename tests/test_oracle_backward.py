@@ -73,3 +73,27 @@ def test_sampled_rows_match_full_backward():
                                            lse[0, :, lo:], keys, q_lo=lo)
     np.testing.assert_allclose(dk_r, dk[0, 0, keys], atol=1e-12)
     np.testing.assert_allclose(dv_r, dv[0, 0, keys], atol=1e-12)
+
+
+def test_stored_output_enters_only_through_D():
+    # Closed form: replacing O by O' in D = rowsum(dO * O) changes dS by -P * dD (dD = D' - D),
+    # so dV is unchanged, dQ changes by -scale * dD_i * sum_j P_ij k_j and dK by
+    # -scale * sum_i dD_i P_ij q_i; giving the exact O reproduces the default (to rounding).
+    q, k, v, do = _inputs(5, 1, 2, 2, 9, 4)
+    o, _ = oracle.attention_full(q, k, v)
+    base = oracle.attention_backward(q, k, v, do)
+    same = oracle.attention_backward(q, k, v, do, o=o)
+    for a, b in zip(base, same):
+        np.testing.assert_allclose(a, b, atol=1e-13)
+    o2 = o + 0.01 * np.random.default_rng(1).standard_normal(o.shape)
+    dq2, dk2, dv2 = oracle.attention_backward(q, k, v, do, o=o2)
+    np.testing.assert_allclose(dv2, base[2], atol=1e-13)
+    scale = 0.5
+    rows = np.arange(9)
+    for h in range(2):
+        s = scale * (q[0, h] @ k[0, h].T)
+        s = np.where(rows[None, :] <= rows[:, None], s, -np.inf)
+        p = np.exp(s - np.log(np.exp(s).sum(axis=1))[:, None])
+        dD = (do[0, h] * (o2[0, h] - o[0, h])).sum(axis=1)
+        np.testing.assert_allclose(dq2[0, h] - base[0][0, h], -scale * dD[:, None] * (p @ k[0, h]), atol=1e-12)
+        np.testing.assert_allclose(dk2[0, h] - base[1][0, h], -scale * (p * dD[:, None]).T @ q[0, h], atol=1e-12)
