@@ -25,6 +25,7 @@
 // Every wait is bounded (WaitCtl): on expiry the kernel records CP_ERR_TIMEOUT with the wait
 // site in the status word, drains its in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
+#include <type_traits>
 #include "sm100.cuh"
 
 namespace cpattn {
@@ -37,6 +38,11 @@ constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: skip the O rescale below 2^8 growth
+#ifndef CPATTN_EMU_PAIRS
+#define CPATTN_EMU_PAIRS 0
+#endif
+// Of every 16 exponential pairs of a 32-column chunk, this many run on the FMA pipe.
+constexpr int kEmuPairs = CPATTN_EMU_PAIRS;
 
 enum WaitSite : int {
   kSiteLoadEmpty = 1, kSiteMmaQ = 2, kSiteMmaKV = 3, kSiteMmaP = 4,
@@ -347,29 +353,37 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int lim = kv_end - kv0;
       if (p.causal) lim = min(lim, q_row - kv0 + 1);
 
-      float s[kBN];
-#pragma unroll
-      for (int cc = 0; cc < kBN / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tS + cc * 32, r);
+      // Row max, then exponentials.  Chunks 0 and 1 of the S row stay in registers from the
+      // max pass; chunks 2 and 3 are re-read from TMEM, each load issued before the previous
+      // chunk's arithmetic so its latency overlaps that work.
+      uint32_t ra[32], rb[32];
+      float m_raw;
+      {
+        uint32_t rc[32], rd[32];
+        tmem_ld32(tS + 0, ra);
+        tmem_ld32(tS + 32, rb);
+        tmem_ld32(tS + 64, rc);
+        tmem_ld32(tS + 96, rd);
         tmem_wait_ld();
+        if (lim < kBN) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[cc * 32 + e] = __uint_as_float(r[e]);
-      }
-      if (lim < kBN) {
+          for (int e = 0; e < 32; ++e) {
+            if (e >= lim) ra[e] = __float_as_uint(-INFINITY);
+            if (32 + e >= lim) rb[e] = __float_as_uint(-INFINITY);
+            if (64 + e >= lim) rc[e] = __float_as_uint(-INFINITY);
+            if (96 + e >= lim) rd[e] = __float_as_uint(-INFINITY);
+          }
+        }
+        float mx0 = fmax3(__uint_as_float(ra[0]), __uint_as_float(rb[0]), __uint_as_float(rc[0]));
+        float mx1 = __uint_as_float(rd[0]);
 #pragma unroll
-        for (int e = 0; e < kBN; ++e)
-          if (e >= lim) s[e] = -INFINITY;
+        for (int e = 1; e < 32; ++e) {
+          mx0 = fmax3(mx0, __uint_as_float(ra[e]), __uint_as_float(rb[e]));
+          mx1 = fmax3(mx1, __uint_as_float(rc[e]), __uint_as_float(rd[e]));
+        }
+        m_raw = fmaxf(mx0, mx1);
       }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-      for (int e = 4; e < kBN; e += 4) {
-        mx0 = fmaxf(mx0, s[e]);
-        mx1 = fmaxf(mx1, s[e + 1]);
-        mx2 = fmaxf(mx2, s[e + 2]);
-        mx3 = fmaxf(mx3, s[e + 3]);
-      }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float m_tile = m_raw * sl2;
       float alpha = 1.f;
       if (m_tile > m_run + kRescaleThreshold) {
         alpha = ex2_approx(m_run - m_tile);  // 0 when m_run = -inf
@@ -377,21 +391,48 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         l_run *= alpha;
       }
       const float m_off = (m_run == -INFINITY) ? 0.f : m_run;
-      float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < kBN / 32; ++cc) {
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m_off, -m_off);
+      uint64_t sum2 = f2_pack(0.f, 0.f);
+      // exponentials of one 32-column chunk -> 16 packed bf16 columns of P (over S columns
+      // already read: P columns [16cc, 16cc+16))
+      auto exp_chunk = [&](const uint32_t (&r)[32], int cc, bool masked) {
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2_approx(fmaf(s[cc * 32 + 2 * e], sl2, -m_off));
-          const float p1 = ex2_approx(fmaf(s[cc * 32 + 2 * e + 1], sl2, -m_off));
-          sum0 += p0;
-          sum1 += p1;
-          pk[e] = pack_bf16x2(p0, p1);
+        for (int e2 = 0; e2 < 16; ++e2) {
+          const int c = cc * 32 + 2 * e2;
+          float s0 = __uint_as_float(r[2 * e2]), s1 = __uint_as_float(r[2 * e2 + 1]);
+          if (masked) {
+            if (c >= lim) s0 = -INFINITY;
+            if (c + 1 >= lim) s1 = -INFINITY;
+          }
+          float x0, x1, p0, p1;
+          f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negm2), x0, x1);
+          if (kEmuPairs > 0 && (e2 * kEmuPairs) % 16 < kEmuPairs) {
+            ex2_fma2(x0, x1, p0, p1);  // this share of the exponentials runs on the FMA pipe
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          sum2 = f2_add(sum2, f2_pack(p0, p1));
+          pk[e2] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + cc * 16, pk);
+      };
+      const bool masked = lim < kBN;  // chunks 0 and 1 were masked in place above
+      exp_chunk(ra, 0, false);
+      tmem_ld32(tS + 64, ra);
+      exp_chunk(rb, 1, false);
+      tmem_wait_ld();
+      tmem_ld32(tS + 96, rb);
+      exp_chunk(ra, 2, masked);
+      tmem_wait_ld();
+      exp_chunk(rb, 3, masked);
+      {
+        float a0, a1;
+        f2_unpack(sum2, a0, a1);
+        l_run += a0 + a1;
       }
-      l_run += sum0 + sum1;
       // O <- alpha * O for rows whose reference max moved (O holds the previous tiles' sum;
       // PV of the previous tile has completed because S of this tile was issued after it).
       if (i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
