@@ -130,6 +130,25 @@ cp_status_t cp_attn_bwd(const cp_plan_t* plan, const cp_tensor_t* q, const cp_te
                         const cp_tensor_t* dout, cp_tensor_t* dq, cp_tensor_t* dk,
                         cp_tensor_t* dv, void* ws, size_t ws_bytes, void* stream);
 
+/* Forward for callers that cannot allocate device memory — for example code running inside
+ * another framework that owns the whole device-memory budget and forbids allocations of its
+ * own, or a host process that reserved all device memory up front.  The pages have no
+ * counterpart to this entry point: it is a deployment variant of cp_attn_fwd.
+ * Same computation and tensors as cp_attn_fwd for ULYSSES and TWO_D plans (RING plans need no
+ * workspace: use cp_attn_fwd; they get CP_ERR_INVALID_ARG here).  Instead of a caller
+ * workspace it uses a scratch array of 64 MiB that the library declares statically: every GPU
+ * that loads the library holds those 64 MiB until the process exits.  Problems whose forward
+ * workspace (cp_attn_workspace_size) exceeds 64 MiB are rejected with CP_ERR_WORKSPACE before
+ * any launch.  The library calls no allocating routine here.  The first call on a device looks
+ * up the scratch's device address (cudaGetSymbolAddress, once per device); make that first
+ * call before any stream capture.  All calls share the one scratch array: calls whose GPU
+ * work overlaps (on different streams, or from different threads) race on it and must be
+ * serialised by the caller.  The scratch keeps the last call's contents; every byte a call
+ * reads is written earlier in the same call.  Device-side wait expiries are not recorded
+ * (there is no status word without an allocation); the waits stay bounded. */
+cp_status_t cp_attn_fwd_noalloc(const cp_plan_t* plan, const cp_tensor_t* q, const cp_tensor_t* k,
+                                const cp_tensor_t* v, cp_tensor_t* o, cp_tensor_t* lse, void* stream);
+
 /* Ulysses all-to-all on one GPU ([CP] §2, [UL] step 2): in [B, L, H, d] (rank s holds rows
  * [s*c, (s+1)*c)) -> out [B, H, L, d] (rank r' holds heads [r'*H/N, (r'+1)*H/N) for all L):
  *     out[b, r'*H/N + h', s*c + t, :] = in[b, s*c + t, r'*H/N + h', :].

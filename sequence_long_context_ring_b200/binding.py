@@ -45,6 +45,7 @@ EXPORTS = [
     "cp_attn_plan", "cp_attn_plan_destroy", "cp_attn_workspace_size", "cp_attn_fwd", "cp_attn_bwd",
     "cp_layout_seq2head", "cp_layout_head2seq", "cp_ring_step", "cp_lse_merge", "cp_device_status",
     "cp_status_string", "cp_plan_step_chunk", "cp_plan_flops", "cp_plan_num_work_items", "cp_version",
+    "cp_attn_fwd_noalloc",
 ]
 
 
@@ -73,6 +74,7 @@ def lib() -> ctypes.CDLL:
             "cp_plan_flops": ([P, ctypes.c_int, ctypes.POINTER(ctypes.c_double)], ctypes.c_int),
             "cp_plan_num_work_items": ([P, ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
             "cp_version": ([], ctypes.c_char_p),
+            "cp_attn_fwd_noalloc": ([P, T, T, T, T, T, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -174,6 +176,15 @@ class Plan:
         td = [tensor_desc(t) for t in (q, k, v, o, lse)]
         _check(lib().cp_attn_fwd(self._h, *[ctypes.byref(t) for t in td], wptr, wlen, _stream(stream)),
                "cp_attn_fwd")
+        return o, lse
+
+    def fwd_noalloc(self, q, k, v, o, lse, stream=None):
+        """Forward of a Ulysses / 2D plan through cp_attn_fwd_noalloc: the library uses its
+        static 64 MiB scratch instead of a workspace and allocates nothing.  o and lse must
+        be given (preallocated by the caller)."""
+        td = [tensor_desc(t) for t in (q, k, v, o, lse)]
+        _check(lib().cp_attn_fwd_noalloc(self._h, *[ctypes.byref(t) for t in td], _stream(stream)),
+               "cp_attn_fwd_noalloc")
         return o, lse
 
     def bwd(self, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, ws=None, stream=None):

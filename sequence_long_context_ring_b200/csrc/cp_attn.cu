@@ -687,3 +687,90 @@ cp_status_t cp_attn_bwd(const cp_plan_t* plan, const cp_tensor_t* q, const cp_te
 }
 
 }  // extern "C"
+
+// =====================================================================================
+// Forward without any device allocation by the library (see cp_attn_fwd_noalloc in
+// cp_attn.h).  Its scratch is this file-scope array; host code reaches it only through the
+// device address that cudaGetSymbolAddress returns for the current device.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB on every device that loads the library
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the static scratch on the current device (looked up once per device).
+cp_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CP_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return CP_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return CP_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return CP_OK;
+}
+
+}  // namespace
+
+extern "C" cp_status_t cp_attn_fwd_noalloc(const cp_plan_t* plan, const cp_tensor_t* q, const cp_tensor_t* k,
+                                           const cp_tensor_t* v, cp_tensor_t* o, cp_tensor_t* lse, void* stream) {
+  if (!plan) return CP_ERR_INVALID_ARG;
+  const cp_attn_config_t& c = plan->cfg;
+  if (c.mode != CP_MODE_ULYSSES && c.mode != CP_MODE_2D) return CP_ERR_INVALID_ARG;
+  CP_TRY(check3(lse, c.B, c.Hq, c.L));
+  CP_TRY(check4(q, CP_BF16, c.B, c.L, c.Hq, c.d));
+  CP_TRY(check4(k, CP_BF16, c.B, c.L, c.Hkv, c.d));
+  CP_TRY(check4(v, CP_BF16, c.B, c.L, c.Hkv, c.d));
+  CP_TRY(check4(o, CP_BF16, c.B, c.L, c.Hq, c.d));
+  size_t need = 0;
+  CP_TRY(cp_attn_workspace_size(plan, 0, &need));
+  if (need > kNoAllocScratchBytes) return CP_ERR_WORKSPACE;  // problem too large for the static scratch
+  void* ws = nullptr;
+  CP_TRY(noalloc_scratch(&ws));
+  const cudaStream_t s = as_stream(stream);
+  const size_t nq = (size_t)c.B * c.Hq * c.L * c.d, nkv = (size_t)c.B * c.Hkv * c.L * c.d;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  void* qh = w;
+  w += align256(nq * 2);
+  void* kh = w;
+  w += align256(nkv * 2);
+  void* vh = w;
+  w += align256(nkv * 2);
+  void* oh = w;
+  // Every byte of the scratch that is read below is written first in this call, so nothing
+  // from an earlier call needs clearing.
+  CP_TRY(seq_to_head_buf(q, qh, s));
+  CP_TRY(seq_to_head_buf(k, kh, s));
+  CP_TRY(seq_to_head_buf(v, vh, s));
+  FwdParams p{};
+  fill_geometry(plan, c.mode == CP_MODE_ULYSSES ? 1 : c.n_cp, p);
+  p.o = oh;
+  p.o_sb = (int64_t)c.Hq * c.L * c.d;
+  p.o_sh = (int64_t)c.L * c.d;
+  p.o_sl = c.d;
+  p.out_fp32 = 0;
+  p.lse = static_cast<float*>(lse->data);
+  p.l_sb = lse->stride[0];
+  p.l_sh = lse->stride[1];
+  p.l_sl = lse->stride[2];
+  p.status = nullptr;  // no status word: it would have to be allocated
+  CUtensorMap mq, mk, mv;
+  CP_TRY(make_map_bhld(&mq, qh, c.B, c.Hq, c.L, c.d, (int64_t)c.Hq * c.L * c.d, (int64_t)c.L * c.d, c.d));
+  CP_TRY(make_map_bhld(&mk, kh, c.B, c.Hkv, c.L, c.d, (int64_t)c.Hkv * c.L * c.d, (int64_t)c.L * c.d, c.d));
+  CP_TRY(make_map_bhld(&mv, vh, c.B, c.Hkv, c.L, c.d, (int64_t)c.Hkv * c.L * c.d, (int64_t)c.L * c.d, c.d));
+  const int64_t grid = (int64_t)p.n_chunks * p.pos_per_chunk * p.n_inner;
+  if (grid > 0) {
+    if (c.d == 128) {
+      CP_TRY(launch_fwd_d<128>(p, mq, mk, mv, grid, s));
+    } else {
+      CP_TRY(launch_fwd_d<64>(p, mq, mk, mv, grid, s));
+    }
+  }
+  return head_buf_to_seq(oh, o, s);
+}
