@@ -174,13 +174,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint8_t* kv_smem = smem + 2 * kTileBytes;                // kStages tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(kv_smem + kStages * kTileBytes);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;                  // [kStages]
-  uint64_t* kv_empty = bars + 1 + kStages;       // [kStages]
-  uint64_t* s_full = bars + 1 + 2 * kStages;     // [2]
-  uint64_t* p_full = bars + 3 + 2 * kStages;     // [2]
-  uint64_t* o_full = bars + 5 + 2 * kStages;
-  uint64_t* drain_bar = bars + 6 + 2 * kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * kStages);
+  // Barriers.  Iteration t uses KV stages 2(t&1) (K_t) and 2(t&1)+1 (V_t).
+  //  kv_full[t&1]  TMA -> MMA: K_t and V_t landed (one wait per iteration)
+  //  kv_free[t&1]  MMA commit after S_B(t): K_t and V_{t-1} are no longer read, and S_B(t) is
+  //                in TMEM (softmax B waits on it too) -- one commit serves both
+  //  s_full_a      MMA commit after S_A(t)
+  //  p_full[ab]    softmax -> MMA: P of tile ab written to TMEM (4 warp arrivals)
+  // A waiter on a two-barrier pair uses parity (t >> 1) & 1; no barrier can run two phases
+  // ahead of its waiter because each next phase needs that waiter's own progress first.
+  uint64_t* kv_full = bars + 1;                  // [2]
+  uint64_t* kv_free = bars + 3;                  // [2]
+  uint64_t* s_full_a = bars + 5;
+  uint64_t* p_full = bars + 6;                   // [2]
+  uint64_t* o_full = bars + 8;
+  uint64_t* drain_bar = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* skip_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -190,12 +198,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_free[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
+    mbar_init(s_full_a, 1);
     mbar_init(&p_full[0], 4);
     mbar_init(&p_full[1], 4);
     mbar_init(o_full, 1);
@@ -235,28 +242,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tma_load_4d(q_smem + kTileBytes + x * kBoxBytes, &tm_q, q_full, x * 64, it.rowB, it.headB, it.b, pol_q);
         }
       }
-      int slot = 0;
-      bool ok = true;
-      for (int i = 0; i < it.n_tiles && ok; ++i) {
+      int issued = 0;
+      for (int i = 0; i < it.n_tiles; ++i) {
+        // K_i and V_i reuse the stages of K_{i-2} and V_{i-2}: both free once the MMAs of
+        // iteration i-1 up to S_B(i-1) have completed (PV_B(i-2) precedes S_B(i-1))
+        if (i >= 2 && !wait_bounded(&kv_free[(i - 1) & 1], ((i - 1) >> 1) & 1, ctl, kSiteLoadEmpty)) break;
         int kv0, kv_end;
         kv_tile(p, it, i, kv0, kv_end);
+        uint64_t* full = &kv_full[i & 1];
+        uint8_t* kdst = kv_smem + (2 * (i & 1)) * kTileBytes;
+        uint8_t* vdst = kdst + kTileBytes;
+        mbar_arrive_expect_tx(full, 2 * kTileBytes);
 #pragma unroll
-        for (int which = 0; which < 2; ++which, ++slot) {
-          const int st = slot % kStages;
-          const uint32_t ph = (slot / kStages) & 1;
-          if (!wait_bounded(&kv_empty[st], ph ^ 1, ctl, kSiteLoadEmpty)) { ok = false; break; }
-          mbar_arrive_expect_tx(&kv_full[st], kTileBytes);
-          const CUtensorMap* tm = which == 0 ? &tm_k : &tm_v;
-          uint8_t* dst = kv_smem + st * kTileBytes;
+        for (int x = 0; x < kBoxes; ++x) tma_load_4d(kdst + x * kBoxBytes, &tm_k, full, x * 64, kv0, it.g, it.b, pol_kv);
 #pragma unroll
-          for (int x = 0; x < kBoxes; ++x)
-            tma_load_4d(dst + x * kBoxBytes, tm, &kv_full[st], x * 64, kv0, it.g, it.b, pol_kv);
-        }
+        for (int x = 0; x < kBoxes; ++x) tma_load_4d(vdst + x * kBoxBytes, &tm_v, full, x * 64, kv0, it.g, it.b, pol_kv);
+        ++issued;
       }
       // drain: every load this thread issued has landed before the CTA can exit
       if (load_q) wait_drain(q_full, 0, ctl);
-      for (int s2 = (slot > kStages ? slot - kStages : 0); s2 < slot; ++s2)
-        wait_drain(&kv_full[s2 % kStages], (s2 / kStages) & 1, ctl);
+      for (int u = (issued > 2 ? issued - 2 : 0); u < issued; ++u) wait_drain(&kv_full[u & 1], (u >> 1) & 1, ctl);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -291,27 +296,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       };
 
+      // TMA-filled operands need no tcgen05 fence (the mbarrier wait orders them); P written
+      // by the softmax threads with tcgen05.st does (after_thread_sync after the wait).
       bool ok = wait_bounded(q_full, 0, ctl, kSiteMmaQ);
-      tc_fence_after();
       const int T = it.n_tiles;
-      int vst_prev = 0;
+      int vst_prev = 1;
       for (int i = 0; i < T && ok; ++i) {
-        const int kslot = 2 * i, vslot = 2 * i + 1;
-        const int kst = kslot % kStages, vst = vslot % kStages;
-        if (!wait_bounded(&kv_full[kst], (kslot / kStages) & 1, ctl, kSiteMmaKV)) { ok = false; break; }
-        tc_fence_after();
+        const int kst = 2 * (i & 1), vst = kst + 1;
+        if (!wait_bounded(&kv_full[i & 1], (i >> 1) & 1, ctl, kSiteMmaKV)) { ok = false; break; }
         issue_s(0, kst);
-        umma_commit(&s_full[0]);
+        umma_commit(s_full_a);
         if (i > 0) {
           if (!wait_bounded(&p_full[1], (i - 1) & 1, ctl, kSiteMmaP)) { ok = false; break; }
           tc_fence_after();
           issue_pv(1, vst_prev, i - 1 > 0);
-          umma_commit(&kv_empty[vst_prev]);
         }
         issue_s(1, kst);
-        umma_commit(&s_full[1]);
-        umma_commit(&kv_empty[kst]);
-        if (!wait_bounded(&kv_full[vst], (vslot / kStages) & 1, ctl, kSiteMmaKV)) { ok = false; break; }
+        umma_commit(&kv_free[i & 1]);
         if (!wait_bounded(&p_full[0], i & 1, ctl, kSiteMmaP)) { ok = false; break; }
         tc_fence_after();
         issue_pv(0, vst, i > 0);
@@ -321,7 +322,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (wait_bounded(&p_full[1], (T - 1) & 1, ctl, kSiteMmaP)) {
           tc_fence_after();
           issue_pv(1, vst_prev, T - 1 > 0);
-          umma_commit(&kv_empty[vst_prev]);
           umma_commit(o_full);
         }
       }
@@ -346,7 +346,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     for (int i = 0; i < it.n_tiles; ++i) {
       // warp-uniform decision: the TMEM loads below are .sync.aligned
-      if (!__all_sync(0xffffffffu, wait_bounded(&s_full[ab], i & 1, ctl, kSiteSoftS))) { ok = false; break; }
+      uint64_t* s_bar = ab == 0 ? s_full_a : &kv_free[i & 1];
+      const uint32_t s_par = ab == 0 ? (i & 1) : ((i >> 1) & 1);
+      if (!__all_sync(0xffffffffu, wait_bounded(s_bar, s_par, ctl, kSiteSoftS))) { ok = false; break; }
       tc_fence_after();
       int kv0, kv_end;
       kv_tile(p, it, i, kv0, kv_end);
