@@ -14,11 +14,14 @@
 // of a finished chunk's partial into the accumulator happens at every chunk boundary as the
 // same rescale-and-add that joins two tiles: (O, LSE) (+) (O', LSE') with weights e^(LSE-m).
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax for tile A (thread t <-> query row t <-> TMEM lane t)
 //   warps 4-7  softmax for tile B
-//   warp  8    TMA producer: Q tiles once, then K_i, V_i into a 4-stage shared-memory ring
+//   warp  8    TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ... into a 5-slot
+//              shared-memory ring (one 128-row K or V tile per slot, each with its own
+//              barrier), issued two iterations ahead of their use
 //   warp  9    MMA issuer (one thread): S = Q K^T into TMEM, O += P V with P read from TMEM
+//   warps 10-11 idle (they complete the producer warpgroup for the register rebalance)
 // TMEM (512 columns x 128 lanes x 32 bit): S_A [0,128) O_A [128,256) S_B [256,384)
 // O_B [384,512).  P (bf16, packed two per column) overwrites the first 64 columns of S.
 //
@@ -32,12 +35,23 @@ namespace cpattn {
 
 constexpr int kBM = 128;       // query rows per tile
 constexpr int kBN = 128;       // keys per KV tile
-constexpr int kStages = 4;     // shared-memory ring, one K or V tile per stage
-constexpr int kFwdThreads = 320;
+constexpr int kKvSlots = 5;    // shared-memory ring: K_i is item 2i, V_i item 2i+1, slot = item % 5
+constexpr int kFwdThreads = 384;  // three warpgroups
+// Registers per thread after the warpgroups rebalance (setmaxnreg): the launch gives every
+// thread 168 (384 x 168 = 64,512 of the SM's 65,536); the producer warpgroup (load, MMA, two
+// idle warps) gives back down to 72 and each softmax warpgroup grows to 216:
+// 2 x 128 x 216 + 128 x 72 = 64,512, the launch's total.  Per SMSP (one warp of each
+// warpgroup): 216 + 216 + 72 = 504 registers x 32 lanes = 16,128 of 16,384.
+constexpr int kSoftmaxRegs = 216;
+constexpr int kProducerRegs = 72;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs <= kFwdThreads * 168, "register split");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: skip the O rescale below 2^8 growth
+// Largest exponent (log2) an unnormalised probability may reach against a row's offset before
+// the offset is moved (and O, l rescaled).
+constexpr float kStaleLimit = 64.0f;
+constexpr float kStaleLimitPow = 18446744073709551616.0f;  // 2^64
 #ifndef CPATTN_EMU_PAIRS
 #define CPATTN_EMU_PAIRS 0
 #endif
@@ -123,30 +137,34 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p) {
   return it;
 }
 
-// i-th KV tile of the item in ring visit order -> first key row and end of its chunk.
-__device__ __forceinline__ void kv_tile(const FwdParams& p, const Item& it, int i, int& kv0, int& kv_end) {
-  int j, tt;
-  if (p.step_rank >= 0) {
-    j = p.step_chunk;
-    tt = i;
-  } else if (p.causal) {
-    if (i < it.n_diag) {
-      j = it.r;
-      tt = i;
+// The KV tiles of an item in ring visit order, walked without divisions (this runs once per
+// tile on the softmax critical path): chunk j, tile tt inside it, tiles left in the chunk.
+//   fused, causal:     chunk r (its first n_diag tiles), then r-1, ..., 0 (all tiles)
+//   fused, non-causal: chunks r, r-1, ... (mod N), all tiles
+//   one ring step:     chunk step_chunk, the item's n_tiles tiles
+struct KvIter {
+  int j, tt, left;
+  __device__ __forceinline__ KvIter(const FwdParams& p, const Item& it) {
+    tt = 0;
+    if (p.step_rank >= 0) {
+      j = p.step_chunk;
+      left = it.n_tiles;
     } else {
-      const int i2 = i - it.n_diag;
-      const int q = i2 / p.tiles_per_chunk;
-      j = it.r - 1 - q;
-      tt = i2 - q * p.tiles_per_chunk;
+      j = it.r;
+      left = p.causal ? it.n_diag : p.tiles_per_chunk;
     }
-  } else {
-    const int s = i / p.tiles_per_chunk;
-    tt = i - s * p.tiles_per_chunk;
-    j = (it.r - s + p.n_chunks) % p.n_chunks;
   }
-  kv0 = j * p.chunk_len + tt * kBN;
-  kv_end = min(j * p.chunk_len + p.chunk_len, p.L);
-}
+  __device__ __forceinline__ void next(const FwdParams& p) {
+    ++tt;
+    if (--left == 0) {
+      tt = 0;
+      left = p.tiles_per_chunk;
+      j = (j == 0 ? p.n_chunks : j) - 1;
+    }
+  }
+  __device__ __forceinline__ int kv0(const FwdParams& p) const { return j * p.chunk_len + tt * kBN; }
+  __device__ __forceinline__ int kv_end(const FwdParams& p) const { return min(j * p.chunk_len + p.chunk_len, p.L); }
+};
 
 // Wait used only while winding down: ignores the abort flag, keeps its own time limit.
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
@@ -171,23 +189,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_smem = smem;                                  // 2 tiles
-  uint8_t* kv_smem = smem + 2 * kTileBytes;                // kStages tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(kv_smem + kStages * kTileBytes);
+  uint8_t* kv_smem = smem + 2 * kTileBytes;                // kKvSlots tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kv_smem + kKvSlots * kTileBytes);
   uint64_t* q_full = bars + 0;
-  // Barriers.  Iteration t uses KV stages 2(t&1) (K_t) and 2(t&1)+1 (V_t).
-  //  kv_full[t&1]  TMA -> MMA: K_t and V_t landed (one wait per iteration)
+  // Barriers.  Ring item n (K_i: n = 2i, V_i: n = 2i+1) lives in slot n % 5.
+  //  kv_full[slot] TMA -> MMA: the item landed (phase parity (n / 5) & 1)
   //  kv_free[t&1]  MMA commit after S_B(t): K_t and V_{t-1} are no longer read, and S_B(t) is
-  //                in TMEM (softmax B waits on it too) -- one commit serves both
+  //                in TMEM (softmax B waits on it too) -- one commit serves both.  The loads
+  //                of iteration t+2 wait for it: K_{t+2} reuses the slot of V_{t-1}, V_{t+2}
+  //                the slot of K_t.
   //  s_full_a      MMA commit after S_A(t)
-  //  p_full[ab]    softmax -> MMA: P of tile ab written to TMEM (4 warp arrivals)
+  //  p_half[ab]    softmax -> MMA: P of keys [0, 64) of tile ab written to TMEM (4 arrivals)
+  //  p_full[ab]    softmax -> MMA: P of keys [64, 128) written (4 warp arrivals)
   // A waiter on a two-barrier pair uses parity (t >> 1) & 1; no barrier can run two phases
   // ahead of its waiter because each next phase needs that waiter's own progress first.
-  uint64_t* kv_full = bars + 1;                  // [2]
-  uint64_t* kv_free = bars + 3;                  // [2]
-  uint64_t* s_full_a = bars + 5;
-  uint64_t* p_full = bars + 6;                   // [2]
-  uint64_t* o_full = bars + 8;
-  uint64_t* drain_bar = bars + 9;
+  uint64_t* kv_full = bars + 1;                  // [kKvSlots]
+  uint64_t* kv_free = bars + 1 + kKvSlots;       // [2]
+  uint64_t* s_full_a = kv_free + 2;
+  uint64_t* p_half = s_full_a + 1;               // [2]
+  uint64_t* p_full = p_half + 2;                 // [2]
+  uint64_t* o_full = p_full + 2;
+  uint64_t* drain_bar = o_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* skip_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -198,13 +220,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_free[s], 1);
-    }
+    for (int s = 0; s < kKvSlots; ++s) mbar_init(&kv_full[s], 1);
+    for (int s = 0; s < 2; ++s) mbar_init(&kv_free[s], 1);
     mbar_init(s_full_a, 1);
-    mbar_init(&p_full[0], 4);
-    mbar_init(&p_full[1], 4);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&p_half[s], 4);
+      mbar_init(&p_full[s], 4);
+    }
     mbar_init(o_full, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -225,6 +247,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const Item it = decode_item(p);
 
+  // Each role branch sets its register budget (warpgroup-wide) and ends at the named barrier
+  // 1 that every warp reaches once its TMEM and shared-memory work is done; warp 0 then frees
+  // TMEM.  The branches never rejoin.
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
   if (warp == kLoadWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
@@ -242,26 +269,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tma_load_4d(q_smem + kTileBytes + x * kBoxBytes, &tm_q, q_full, x * 64, it.rowB, it.headB, it.b, pol_q);
         }
       }
-      int issued = 0;
-      for (int i = 0; i < it.n_tiles; ++i) {
-        // K_i and V_i reuse the stages of K_{i-2} and V_{i-2}: both free once the MMAs of
-        // iteration i-1 up to S_B(i-1) have completed (PV_B(i-2) precedes S_B(i-1))
-        if (i >= 2 && !wait_bounded(&kv_free[(i - 1) & 1], ((i - 1) >> 1) & 1, ctl, kSiteLoadEmpty)) break;
-        int kv0, kv_end;
-        kv_tile(p, it, i, kv0, kv_end);
-        uint64_t* full = &kv_full[i & 1];
-        uint8_t* kdst = kv_smem + (2 * (i & 1)) * kTileBytes;
-        uint8_t* vdst = kdst + kTileBytes;
-        mbar_arrive_expect_tx(full, 2 * kTileBytes);
+      int issued = 0;  // ring items issued
+      KvIter kvi(p, it);
+      for (int i = 0; i < it.n_tiles; ++i, kvi.next(p)) {
+        // K_i and V_i take the slots of V_{i-3} and K_{i-2}: both free once the MMAs of
+        // iteration i-2 up to S_B(i-2) have completed (PV_B(i-3) precedes S_B(i-2))
+        if (i >= 2 && !wait_bounded(&kv_free[i & 1], ((i - 2) >> 1) & 1, ctl, kSiteLoadEmpty)) break;
+        const int kv0 = kvi.kv0(p);
 #pragma unroll
-        for (int x = 0; x < kBoxes; ++x) tma_load_4d(kdst + x * kBoxBytes, &tm_k, full, x * 64, kv0, it.g, it.b, pol_kv);
+        for (int kv = 0; kv < 2; ++kv) {
+          const int n = 2 * i + kv;
+          uint64_t* full = &kv_full[n % kKvSlots];
+          uint8_t* dst = kv_smem + (n % kKvSlots) * kTileBytes;
+          mbar_arrive_expect_tx(full, kTileBytes);
 #pragma unroll
-        for (int x = 0; x < kBoxes; ++x) tma_load_4d(vdst + x * kBoxBytes, &tm_v, full, x * 64, kv0, it.g, it.b, pol_kv);
-        ++issued;
+          for (int x = 0; x < kBoxes; ++x)
+            tma_load_4d(dst + x * kBoxBytes, kv == 0 ? &tm_k : &tm_v, full, x * 64, kv0, it.g, it.b, pol_kv);
+        }
+        issued += 2;
       }
-      // drain: every load this thread issued has landed before the CTA can exit
+      // drain: every load this thread issued has landed before the CTA can exit (the last
+      // fill of each slot is the only phase of its barrier still pending)
       if (load_q) wait_drain(q_full, 0, ctl);
-      for (int u = (issued > 2 ? issued - 2 : 0); u < issued; ++u) wait_drain(&kv_full[u & 1], (u >> 1) & 1, ctl);
+      for (int n = (issued > kKvSlots ? issued - kKvSlots : 0); n < issued; ++n)
+        wait_drain(&kv_full[n % kKvSlots], (n / kKvSlots) & 1, ctl);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -284,53 +315,58 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                   kk > 0 ? 1u : 0u);
         }
       };
-      // O_ab += P_ab V: A = P from TMEM (8 columns per 16 keys), B = V N-major (d contiguous)
-      auto issue_pv = [=](int ab, int st, bool acc) {
+      // O_ab += P_ab V over keys [64 h, 64 h + 64): A = P from TMEM (8 columns per 16 keys),
+      // B = V N-major (d contiguous)
+      auto issue_pv = [=](int ab, int st, int h, bool acc) {
         const uint32_t vaddr = kv_addr0 + st * kTileBytes;
         const uint32_t p_tmem = tmem_base + ab * 256;
         const uint32_t o_tmem = tmem_base + 128 + ab * 256;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
           umma_ts(o_tmem, p_tmem + kk * 8, make_sdesc(vaddr + kk * 2048, kBoxBytes, 1024), idesc_o,
                   (acc || kk > 0) ? 1u : 0u);
         }
+      };
+      // both halves of PV_ab, each after its half of P is in TMEM
+      auto wait_issue_pv = [&](int ab, int st, int t) {
+        if (!wait_bounded(&p_half[ab], t & 1, ctl, kSiteMmaP)) return false;
+        tc_fence_after();
+        issue_pv(ab, st, 0, t > 0);
+        if (!wait_bounded(&p_full[ab], t & 1, ctl, kSiteMmaP)) return false;
+        tc_fence_after();
+        issue_pv(ab, st, 1, true);
+        return true;
       };
 
       // TMA-filled operands need no tcgen05 fence (the mbarrier wait orders them); P written
       // by the softmax threads with tcgen05.st does (after_thread_sync after the wait).
       bool ok = wait_bounded(q_full, 0, ctl, kSiteMmaQ);
       const int T = it.n_tiles;
-      int vst_prev = 1;
+      int vslot_prev = 0;
       for (int i = 0; i < T && ok; ++i) {
-        const int kst = 2 * (i & 1), vst = kst + 1;
-        if (!wait_bounded(&kv_full[i & 1], (i >> 1) & 1, ctl, kSiteMmaKV)) { ok = false; break; }
-        issue_s(0, kst);
+        const int nk = 2 * i, nv = 2 * i + 1;
+        const int kslot = nk % kKvSlots, vslot = nv % kKvSlots;
+        if (!wait_bounded(&kv_full[kslot], (nk / kKvSlots) & 1, ctl, kSiteMmaKV)) { ok = false; break; }
+        issue_s(0, kslot);
         umma_commit(s_full_a);
-        if (i > 0) {
-          if (!wait_bounded(&p_full[1], (i - 1) & 1, ctl, kSiteMmaP)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(1, vst_prev, i - 1 > 0);
-        }
-        issue_s(1, kst);
+        if (i > 0 && !wait_issue_pv(1, vslot_prev, i - 1)) { ok = false; break; }
+        issue_s(1, kslot);
         umma_commit(&kv_free[i & 1]);
-        if (!wait_bounded(&p_full[0], i & 1, ctl, kSiteMmaP)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(0, vst, i > 0);
-        vst_prev = vst;
+        if (!wait_bounded(&kv_full[vslot], (nv / kKvSlots) & 1, ctl, kSiteMmaKV)) { ok = false; break; }
+        if (!wait_issue_pv(0, vslot, i)) { ok = false; break; }
+        vslot_prev = vslot;
       }
-      if (ok && T > 0) {
-        if (wait_bounded(&p_full[1], (T - 1) & 1, ctl, kSiteMmaP)) {
-          tc_fence_after();
-          issue_pv(1, vst_prev, T - 1 > 0);
-          umma_commit(o_full);
-        }
-      }
+      if (ok && T > 0 && wait_issue_pv(1, vslot_prev, T - 1)) umma_commit(o_full);
       // drain: all MMAs issued by this thread are complete before TMEM is freed
       umma_commit(drain_bar);
       wait_drain(drain_bar, 0, ctl);
     }
     __syncwarp();
+  }
+  tc_fence_before();
+  asm volatile("bar.sync 1, %0;" ::"n"(kFwdThreads) : "memory");
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ---------------- softmax / correction / epilogue (warps 0-7) ----------------
     const int ab = warp >> 2;                       // 0: tile A, 1: tile B
     const uint32_t lane_base = (warp & 3) * 32;     // TMEM lane window of this warp
@@ -340,105 +376,146 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tS = tmem_base + (ab ? 256u : 0u) + (lane_base << 16);
     const uint32_t tO = tmem_base + (ab ? 384u : 128u) + (lane_base << 16);
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY;  // running max of scaled scores, log2 units
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    // Exponent offset of the row (log2 units of the scaled scores): the exact max of the first
+    // tile, then kept.  Exponentials are 2^(s*sl2 - m_run); while they stay below 2^kStaleLimit
+    // nothing overflows (O, l < 2^(64+18+16) in fp32) and the result is exact, because the
+    // final normalisation and the LSE use the same offset.  A tile that would pass the limit
+    // moves the offset to its own max and rescales O and l by 2^(old - new).
+    float m_run = -INFINITY;
     float l_run = 0.f;        // running sum of 2^(s*sl2 - m_run)
     bool ok = true;
 
-    for (int i = 0; i < it.n_tiles; ++i) {
-      // warp-uniform decision: the TMEM loads below are .sync.aligned
-      uint64_t* s_bar = ab == 0 ? s_full_a : &kv_free[i & 1];
-      const uint32_t s_par = ab == 0 ? (i & 1) : ((i >> 1) & 1);
-      if (!__all_sync(0xffffffffu, wait_bounded(s_bar, s_par, ctl, kSiteSoftS))) { ok = false; break; }
-      tc_fence_after();
-      int kv0, kv_end;
-      kv_tile(p, it, i, kv0, kv_end);
-      int lim = kv_end - kv0;
-      if (p.causal) lim = min(lim, q_row - kv0 + 1);
-
-      // Row max, then exponentials.  Chunks 0 and 1 of the S row stay in registers from the
-      // max pass; chunks 2 and 3 are re-read from TMEM, each load issued before the previous
-      // chunk's arithmetic so its latency overlaps that work.
-      uint32_t ra[32], rb[32];
-      float m_raw;
-      {
-        uint32_t rc[32], rd[32];
-        tmem_ld32(tS + 0, ra);
-        tmem_ld32(tS + 32, rb);
-        tmem_ld32(tS + 64, rc);
-        tmem_ld32(tS + 96, rd);
-        tmem_wait_ld();
-        if (lim < kBN) {
+    // Masked key columns (c >= lim) of one 32-column chunk of the S row -> -inf.
+    auto mask_chunk = [](uint32_t (&r)[32], int c0, int lim) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (e >= lim) ra[e] = __float_as_uint(-INFINITY);
-            if (32 + e >= lim) rb[e] = __float_as_uint(-INFINITY);
-            if (64 + e >= lim) rc[e] = __float_as_uint(-INFINITY);
-            if (96 + e >= lim) rd[e] = __float_as_uint(-INFINITY);
-          }
-        }
-        float mx0 = fmax3(__uint_as_float(ra[0]), __uint_as_float(rb[0]), __uint_as_float(rc[0]));
-        float mx1 = __uint_as_float(rd[0]);
+      for (int e = 0; e < 32; ++e)
+        if (c0 + e >= lim) r[e] = __float_as_uint(-INFINITY);
+    };
+    // Row max of one chunk as two interleaved 3-input chains (depth 8 each).
+    auto max_chunk = [](const uint32_t (&r)[32]) {
+      float a = fmax3(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
+      float b = fmax3(__uint_as_float(r[3]), __uint_as_float(r[4]), __uint_as_float(r[5]));
 #pragma unroll
-        for (int e = 1; e < 32; ++e) {
-          mx0 = fmax3(mx0, __uint_as_float(ra[e]), __uint_as_float(rb[e]));
-          mx1 = fmax3(mx1, __uint_as_float(rc[e]), __uint_as_float(rd[e]));
-        }
-        m_raw = fmaxf(mx0, mx1);
+      for (int e = 6; e < 30; e += 4) {
+        a = fmax3(a, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+        b = fmax3(b, __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
       }
-      const float m_tile = m_raw * sl2;
-      float alpha = 1.f;
-      if (m_tile > m_run + kRescaleThreshold) {
-        alpha = ex2_approx(m_run - m_tile);  // 0 when m_run = -inf
-        m_run = m_tile;
-        l_run *= alpha;
-      }
-      const float m_off = (m_run == -INFINITY) ? 0.f : m_run;
-      const uint64_t sl2x2 = f2_pack(sl2, sl2);
-      const uint64_t negm2 = f2_pack(-m_off, -m_off);
+      return fmax3(a, b, fmaxf(__uint_as_float(r[30]), __uint_as_float(r[31])));
+    };
+    // 2^(s*sl2 - m) of one 32-column chunk -> 16 packed bf16 columns of P written over S
+    // columns already read (P columns [16cc, 16cc+16)); returns the chunk's sum.  emu: a share
+    // of the pairs runs on the FMA pipe (only for chunks without masked columns, whose
+    // exponentials must be exact zeros).
+    auto exp_chunk = [&](const uint32_t (&r)[32], int cc, uint64_t negm2, bool emu) {
       uint64_t sum2 = f2_pack(0.f, 0.f);
-      // exponentials of one 32-column chunk -> 16 packed bf16 columns of P (over S columns
-      // already read: P columns [16cc, 16cc+16))
-      auto exp_chunk = [&](const uint32_t (&r)[32], int cc, bool masked) {
-        uint32_t pk[16];
 #pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          const int c = cc * 32 + 2 * e2;
-          float s0 = __uint_as_float(r[2 * e2]), s1 = __uint_as_float(r[2 * e2 + 1]);
-          if (masked) {
-            if (c >= lim) s0 = -INFINITY;
-            if (c + 1 >= lim) s1 = -INFINITY;
-          }
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int e2 = h * 8 + e;
           float x0, x1, p0, p1;
-          f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negm2), x0, x1);
-          if (kEmuPairs > 0 && (e2 * kEmuPairs) % 16 < kEmuPairs) {
-            ex2_fma2(x0, x1, p0, p1);  // this share of the exponentials runs on the FMA pipe
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * e2]), __uint_as_float(r[2 * e2 + 1])), sl2x2, negm2), x0,
+                    x1);
+          if (kEmuPairs > 0 && emu && (e2 * kEmuPairs) % 16 < kEmuPairs) {
+            ex2_fma2(x0, x1, p0, p1);
           } else {
             p0 = ex2_approx(x0);
             p1 = ex2_approx(x1);
           }
           sum2 = f2_add(sum2, f2_pack(p0, p1));
-          pk[e2] = pack_bf16x2(p0, p1);
+          pk[e] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tS + cc * 16, pk);
-      };
-      const bool masked = lim < kBN;  // chunks 0 and 1 were masked in place above
-      exp_chunk(ra, 0, false);
-      tmem_ld32(tS + 64, ra);
-      exp_chunk(rb, 1, false);
-      tmem_wait_ld();
-      tmem_ld32(tS + 96, rb);
-      exp_chunk(ra, 2, masked);
-      tmem_wait_ld();
-      exp_chunk(rb, 3, masked);
-      {
-        float a0, a1;
-        f2_unpack(sum2, a0, a1);
-        l_run += a0 + a1;
+        tmem_st8(tS + cc * 16 + h * 8, pk);
       }
-      // O <- alpha * O for rows whose reference max moved (O holds the previous tiles' sum;
-      // PV of the previous tile has completed because S of this tile was issued after it).
-      if (i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
+      float a0, a1;
+      f2_unpack(sum2, a0, a1);
+      return a0 + a1;
+    };
+    // all stores of this thread's P are in TMEM before one lane of the warp arrives
+    auto publish = [&](uint64_t* bar) {
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+
+    KvIter kvi(p, it);
+    for (int i = 0; i < it.n_tiles; ++i, kvi.next(p)) {
+      // warp-uniform decisions only: the TMEM loads and stores below are .sync.aligned
+      uint64_t* s_bar = ab == 0 ? s_full_a : &kv_free[i & 1];
+      const uint32_t s_par = ab == 0 ? (i & 1) : ((i >> 1) & 1);
+      if (!__all_sync(0xffffffffu, wait_bounded(s_bar, s_par, ctl, kSiteSoftS))) { ok = false; break; }
+      tc_fence_after();
+      const int kv0 = kvi.kv0(p);
+      int lim = kvi.kv_end(p) - kv0;
+      if (p.causal) lim = min(lim, q_row - kv0 + 1);
+      const bool masked = __any_sync(0xffffffffu, lim < kBN);
+      const bool emu = !masked;
+
+      // The whole S row stays in registers until the tile is settled (a rare recompute needs
+      // it; P overwrites the first 64 columns of S in TMEM).  Chunks 2 and 3 load while the
+      // exponentials of chunks 0 and 1 run.
+      uint32_t ra[32], rb[32], rc[32], rd[32];
+      tmem_ld32(tS + 0, ra);
+      tmem_ld32(tS + 32, rb);
+      tmem_wait_ld();
+      tmem_ld32(tS + 64, rc);
+      tmem_ld32(tS + 96, rd);
+      if (masked) {
+        mask_chunk(ra, 0, lim);
+        mask_chunk(rb, 32, lim);
+      }
+      if (i == 0) {
+        // first tile: the exact row max before any exponential
+        tmem_wait_ld();
+        if (masked) {
+          mask_chunk(rc, 64, lim);
+          mask_chunk(rd, 96, lim);
+        }
+        m_run = fmaxf(fmaxf(max_chunk(ra), max_chunk(rb)), fmaxf(max_chunk(rc), max_chunk(rd))) * sl2;
+      }
+      uint64_t negm2;
+      {
+        const float m_off = (m_run == -INFINITY) ? 0.f : m_run;
+        negm2 = f2_pack(-m_off, -m_off);
+      }
+      float l_tile = exp_chunk(ra, 0, negm2, emu);
+      l_tile += exp_chunk(rb, 1, negm2, emu);
+      if (i > 0) {
+        tmem_wait_ld();
+        if (masked) {
+          mask_chunk(rc, 64, lim);
+          mask_chunk(rd, 96, lim);
+        }
+      }
+      // Before the first half of P is released: the offset must keep every exponential of the
+      // tile below 2^kStaleLimit (keys [0,64) by their sum, [64,128) by their max).
+      const float m23 = fmaxf(max_chunk(rc), max_chunk(rd)) * sl2;
+      const bool over = !(l_tile <= kStaleLimitPow) || m23 > m_run + kStaleLimit;
+      if (__any_sync(0xffffffffu, over)) {
+        // rare: move the offset of the rows that need it to their tile max, rescale O and l
+        // (O holds the previous tiles' sum: PV of the previous tile has completed because S of
+        // this tile was issued after it), and recompute the whole tile's P; rows whose offset
+        // did not move recompute the same values
+        float alpha = 1.f;
+        if (over) {
+          const float m_new = fmaxf(fmaxf(max_chunk(ra), max_chunk(rb)) * sl2, m23);
+          if (m_new > m_run) {
+            alpha = ex2_approx(m_run - m_new);  // 0 when m_run = -inf
+            m_run = m_new;
+          }
+        }
+        const float m_off = (m_run == -INFINITY) ? 0.f : m_run;
+        negm2 = f2_pack(-m_off, -m_off);
+        tmem_wait_st();
+        l_tile = exp_chunk(ra, 0, negm2, false);
+        l_tile += exp_chunk(rb, 1, negm2, false);
+        l_tile += exp_chunk(rc, 2, negm2, false);
+        l_tile += exp_chunk(rd, 3, negm2, false);
+        l_run = l_run * alpha + l_tile;
+#pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t r[32];
           tmem_ld32(tO + cc * 32, r);
@@ -447,11 +524,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
           tmem_st32(tO + cc * 32, r);
         }
+        publish(&p_half[ab]);
+        publish(&p_full[ab]);
+      } else {
+        publish(&p_half[ab]);
+        l_tile += exp_chunk(rc, 2, negm2, emu);
+        l_tile += exp_chunk(rd, 3, negm2, emu);
+        l_run += l_tile;
+        publish(&p_full[ab]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[ab]);
     }
 
     // ---------------- epilogue: O / l, LSE ----------------
@@ -494,19 +575,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         p.lse[it.b * p.l_sb + head * p.l_sh + orow * p.l_sl] = lse;
       }
     }
-  }
 
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"n"(kFwdThreads) : "memory");
+    if (warp == 0) {
+      tc_fence_after();
+      tmem_dealloc(tmem_base, kTmemCols);
+    }
   }
 }
 
-// Dynamic shared memory: 1 KB alignment slack + Q (2 tiles) + KV ring + barriers.
+// Dynamic shared memory: 1 KB alignment slack + Q (2 tiles) + KV ring + barriers
+// (d = 128: 230,656 bytes of the 232,448 a CTA may use).
 __host__ __device__ constexpr size_t fwd_smem_bytes(int d) {
-  return 1024 + static_cast<size_t>(2 + kStages) * 128 * d * 2 + 256;
+  return 1024 + static_cast<size_t>(2 + kKvSlots) * 128 * d * 2 + 256;
 }
 
 }  // namespace cpattn
