@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU work of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements of the other hot-path steps")
+    ap.add_argument("--rows-only", action="store_true", help="measure only the other hot-path steps (one JSON line)")
+    ap.add_argument("--rows-l-div", type=int, default=1, help="divide each row's sequence length (small ncu cases)")
     return ap.parse_args()
 
 
@@ -212,6 +215,126 @@ def run_reference(args, w):
 
 
 # ------------------------------------------------------------------------------------------
+def _time_ms(fn, stream, warmup=3, reps=10):
+    """Median device time of fn() (CUDA events on `stream`, synchronised on both sides)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    ev[0].record(stream)
+    for i in range(reps):
+        fn()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(reps))
+
+
+def measure_rows(dev, peaks, l_div: int = 1):
+    """Device time of every other step of the hot path at its workload's shape (random bf16
+    device inputs; no host data): the Ulysses permutes and the Ulysses forward (c4 shape), the
+    2D forward and backward (c5 shape), the ring backward (c2 shape), and one step-wise ring
+    step plus its LSE merge (c2 shape).  Each entry carries its roofline: HBM-bound steps
+    against the measured copy bandwidth, contractions against the measured bf16 peak."""
+    import torch
+    from sequence_long_context_ring_b200 import binding
+    from sequence_long_context_ring_b200.binding import Plan
+    from sequence_long_context_ring_b200.configs import WORKLOADS
+
+    hbm = float(peaks["hbm_gbs"])
+    tc = float(peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained")))
+    stream = torch.cuda.current_stream(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(2024)
+    rows = {}
+
+    def rnd(*shape):
+        return torch.randn(shape, device=dev, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+    def hbm_row(name, workload, ms, nbytes):
+        gbs = nbytes / (ms / 1e3) / 1e9
+        rows[name] = {"workload": workload, "ms": ms, "value": gbs, "unit": "GB/s",
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                                   "bytes": nbytes}}
+
+    def tc_row(name, workload, ms, flops):
+        tf = flops / (ms / 1e3) / 1e12
+        rows[name] = {"workload": workload, "ms": ms, "value": tf, "unit": "TFLOP/s",
+                      "roofline": {"bound": "tensor", "achieved": tf, "peak": tc, "unit": "TFLOP/s", "frac": tf / tc,
+                                   "flops": flops}}
+
+    # a4 / a5: Ulysses re-layout at the c4 shape (one 1 GiB tensor each way)
+    w = WORKLOADS["c4"]
+    L = w.L // l_div
+    x = rnd(w.B, L, w.Hq, w.d)
+    y = torch.empty((w.B, w.Hq, L, w.d), dtype=torch.bfloat16, device=dev)
+    nbytes = 2 * x.numel() * 2
+    hbm_row("seq2head", f"c4 shape [1,{L},32,128] bf16", _time_ms(lambda: binding.seq2head(w.n_cp, x, y), stream), nbytes)
+    hbm_row("head2seq", f"c4 shape [1,32,{L},128] bf16", _time_ms(lambda: binding.head2seq(w.n_cp, y, x), stream), nbytes)
+    del y
+    # a6: Ulysses forward, c4 (seq->head, attention per head group, head->seq)
+    k, v = rnd(w.B, L, w.Hkv, w.d), rnd(w.B, L, w.Hkv, w.d)
+    plan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp, mode="ulysses")
+    o = torch.empty_like(x)
+    lse = torch.empty((w.B, w.Hq, L), dtype=torch.float32, device=dev)
+    ws = plan.workspace(False, dev)
+    tc_row("ulysses_fwd", f"c4 L={L} degree 8", _time_ms(lambda: plan.fwd(x, k, v, o, lse, ws, stream), stream, reps=5),
+           plan.flops(False))
+    del x, k, v, o, lse, ws, plan
+    # 2D forward and backward, c5
+    w = WORKLOADS["c5"]
+    L = w.L // l_div
+    q, k, v, do = rnd(w.B, L, w.Hq, w.d), rnd(w.B, L, w.Hkv, w.d), rnd(w.B, L, w.Hkv, w.d), rnd(w.B, L, w.Hq, w.d)
+    plan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp, n_hp=w.n_hp, mode="2d")
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, L), dtype=torch.float32, device=dev)
+    ws = plan.workspace(False, dev)
+    tc_row("2d_fwd", f"c5 L={L} grid 4x4", _time_ms(lambda: plan.fwd(q, k, v, o, lse, ws, stream), stream, reps=5),
+           plan.flops(False))
+    wsb = plan.workspace(True, dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    tc_row("2d_bwd", f"c5 L={L} grid 4x4 (D preprocess, a2a of q/k/v/dO, kernel, dQ cast, a2a back)",
+           _time_ms(lambda: plan.bwd(q, k, v, o, lse, do, dq, dk, dv, wsb, stream), stream, reps=5), plan.flops(True))
+    del q, k, v, do, o, lse, ws, wsb, dq, dk, dv, plan
+    # ring backward and the step-wise path at the c2 shape
+    w = WORKLOADS["c2"]
+    L = w.L // l_div
+    q, k, v, do = rnd(w.B, w.Hq, L, w.d), rnd(w.B, w.Hkv, L, w.d), rnd(w.B, w.Hkv, L, w.d), rnd(w.B, w.Hq, L, w.d)
+    plan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp)
+    o, lse = plan.fwd(q, k, v)
+    wsb = plan.workspace(True, dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    tc_row("ring_bwd", f"c2 L={L} N=8 (D preprocess, kernel, dQ cast)",
+           _time_ms(lambda: plan.bwd(q, k, v, o, lse, do, dq, dk, dv, wsb, stream), stream, reps=5), plan.flops(True))
+    ch = L // w.n_cp
+    po = torch.empty((w.B, w.Hq, ch, w.d), dtype=torch.float32, device=dev)
+    pl = torch.empty((w.B, w.Hq, ch), dtype=torch.float32, device=dev)
+    r = w.n_cp - 1
+    tc_row("ring_step", f"c2 rank {r} step 1 (full chunk {r - 1} of {ch} keys)",
+           _time_ms(lambda: plan.ring_step(r, 1, q, k, v, po, pl, stream), stream),
+           4.0 * w.B * w.Hq * w.d * ch * ch)
+    acc_o = torch.zeros_like(po)
+    acc_l = torch.full_like(pl, -float("inf"))
+    hbm_row("lse_merge", f"c2 chunk [1,32,{ch},128] fp32",
+            _time_ms(lambda: binding.lse_merge(acc_o, acc_l, po, pl, stream), stream),
+            (3 * po.numel() + 3 * pl.numel()) * 4)
+    torch.cuda.synchronize()
+    st, word = plan.device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) in the row measurements")
+    return rows
+
+
+def run_rows_only(args):
+    import torch
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    peaks, src = load_peaks()
+    rows = measure_rows(dev, peaks, args.rows_l_div)
+    print(json.dumps({"rows": rows, "peaks": src, "rows_l_div": args.rows_l_div}), flush=True)
+    return 0
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -319,6 +442,11 @@ def run_ours(args, w):
                 "peak_source": f"{peak_src} bf16_tflops_sustained (seconds-long back-to-back launches)"}
     launches = args.steps * (1 if w.mode == "ring" else 5)
 
+    row_meas = None
+    if world == 1 and not args.no_rows:
+        del qd, kd, vd, qh, kh, vh, oh, lh
+        row_meas = measure_rows(dev, peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
@@ -347,6 +475,7 @@ def run_ours(args, w):
                     "steps": args.e2e_steps},
             "gpu_launches": launches,
             "clocks": clk,
+            "rows": row_meas,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -361,6 +490,8 @@ def main():
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.rows_only:
+        return run_rows_only(args)
     return run_ours(args, w)
 
 
