@@ -1,5 +1,5 @@
 // aux_kernels.cuh — HBM-bound kernels: Ulysses re-layout, step-wise LSE merge, and the
-// backward's D = rowsum(dO * O) preprocess and dQ fp32 -> bf16 conversion.
+// backward's D = rowsum(dO * O) preprocess.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -142,35 +142,6 @@ __global__ void __launch_bounds__(256) rowdot_kernel(const DotParams p) {
   }
   for (int off = lpr >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (live && vec == 0) p.D[b * p.D_sb + h * p.D_sh + l * p.D_sl] = acc;
-}
-
-// ---- dQ accumulator (fp32) * scale -> bf16 output ------------------------------------
-struct CastParams {
-  const float* src;      // contiguous [B, H, L, d]
-  __nv_bfloat16* dst;
-  float scale;           // applied before rounding
-  int B, H, L, d;
-  long long d_sb, d_sh, d_sl;
-};
-
-__global__ void __launch_bounds__(256) cast_bf16_kernel(const CastParams p) {
-  const long long n4 = static_cast<long long>(p.B) * p.H * p.L * p.d / 4;
-  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n4) return;
-  const long long e = i * 4;
-  const int c = static_cast<int>(e % p.d);
-  long long t = e / p.d;
-  const int l = static_cast<int>(t % p.L);
-  t /= p.L;
-  const int h = static_cast<int>(t % p.H);
-  const int b = static_cast<int>(t / p.H);
-  const float4 v = reinterpret_cast<const float4*>(p.src)[i];
-  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x * p.scale, v.y * p.scale);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(v.z * p.scale, v.w * p.scale);
-  uint2 packed;
-  packed.x = *reinterpret_cast<uint32_t*>(&lo);
-  packed.y = *reinterpret_cast<uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(p.dst + b * p.d_sb + h * p.d_sh + l * p.d_sl + c) = packed;
 }
 
 // ---- fill a step-wise partial with the merge identity (O = 0, LSE = -inf) -------------------

@@ -1,0 +1,392 @@
+// bwd_dq_kernel.cuh — dQ of the ring-attention backward for sm_100a (tcgen05 + TMEM + TMA),
+// query-stationary, recomputing the probabilities from the forward's stored LSE
+// ("スケーラビリティとメモリ管理" in "長いシーケンスのLLMトレーニングの進展": keep only what
+// is needed, recompute the rest).  For one 128-row query tile of head h, over every KV tile it
+// sees, in ring order (its own chunk r first, then r-1, ..., 0; non-causal: all chunks):
+//   S = Q K^T;  P = 2^(S*scale*log2e - LSE*log2e);  dP = dO V^T;  dS = P o (dP - D);
+//   dQ += dS K      (D = rowsum(dO o O) from the preprocess kernel)
+// dQ accumulates in TMEM over the whole visit and is written once, scaled and rounded to
+// bf16: no atomics, and the result does not depend on the order in which CTAs run.
+//
+// Warp roles (192 threads):
+//   warps 0-3  elementwise: thread t <-> query row t <-> TMEM lane t; epilogue writes dQ
+//   warp  4    loads: Q and dO once; K_i into a 3-slot ring, V_i into a 2-slot ring (TMA)
+//   warp  5    MMA issuer (one thread)
+// TMEM columns: dQ [0,128)  S buffer 0 [128,256)  S buffer 1 [256,384)  dP [384,512).
+// S(i) goes to buffer i&1; dS(i) (bf16, two per column) overwrites the first 64 columns of it.
+// Per iteration the MMA issues S(i+1) and dP(i+1) before dQ += dS(i) K(i), so the tensor pipe
+// computes the next tile's products while the elementwise warps work on this one.
+#pragma once
+#include "sm100.cuh"
+
+namespace cpattn {
+
+constexpr int kDqThreads = 192;
+constexpr int kDqLoadWarp = 4;
+constexpr int kDqMmaWarp = 5;
+constexpr int kDqKSlots = 3;
+constexpr int kDqVSlots = 2;
+
+enum DqSite : int {
+  kQSiteLoadK = 33, kQSiteLoadV = 34, kQSiteMmaQ = 35, kQSiteMmaK = 36, kQSiteMmaV = 37, kQSiteMmaDpFree = 38,
+  kQSiteMmaDs = 39, kQSiteS = 40, kQSiteDp = 41, kQSiteDone = 42, kQSiteDrain = 43,
+};
+
+struct DqParams {
+  int B, Hq, Hkv, L, d, G;
+  int n_chunks, chunk_len, tiles_per_chunk;
+  int causal;
+  float scale;        // softmax scale (applied to dQ once, in the epilogue)
+  float scale_log2;   // scale * log2(e)
+  const float* lse;   // [B, Hq, L] natural-log LSE of the forward
+  long long lse_sb, lse_sh, lse_sl;
+  const float* Dvec;  // [B, Hq, L] rowsum(dO * O), contiguous
+  __nv_bfloat16* dq;  // [B, Hq, L, d] by the strides below
+  long long dq_sb, dq_sh, dq_sl;
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+
+struct DqItem {
+  int b, h, g, r, row0, q_end, n_diag, n_tiles;
+};
+
+// Work items longest first: last chunk, last query tiles (the causal work grows with the row).
+__device__ __forceinline__ DqItem decode_dq_item(const DqParams& p) {
+  DqItem it;
+  const int n_inner = p.B * p.Hq;
+  const int pos = blockIdx.x / n_inner;
+  const int inner = blockIdx.x - pos * n_inner;
+  it.b = inner / p.Hq;
+  it.h = inner - it.b * p.Hq;
+  it.g = it.h / p.G;
+  it.r = p.n_chunks - 1 - pos / p.tiles_per_chunk;
+  const int qpos = p.tiles_per_chunk - 1 - pos % p.tiles_per_chunk;
+  const int c0 = it.r * p.chunk_len;
+  it.row0 = c0 + qpos * 128;
+  it.q_end = min(c0 + p.chunk_len, p.L);
+  it.n_diag = qpos + 1;  // tiles of chunk r up to (and including) the one holding the diagonal
+  it.n_tiles = p.causal ? it.n_diag + it.r * p.tiles_per_chunk : p.n_chunks * p.tiles_per_chunk;
+  return it;
+}
+
+// KV tiles of the item in ring visit order, without divisions: chunk j, tile tt, tiles left.
+struct DqKvIter {
+  int j, tt, left;
+  __device__ __forceinline__ DqKvIter(const DqParams& p, const DqItem& it)
+      : j(it.r), tt(0), left(p.causal ? it.n_diag : p.tiles_per_chunk) {}
+  __device__ __forceinline__ void next(const DqParams& p) {
+    ++tt;
+    if (--left == 0) {
+      tt = 0;
+      left = p.tiles_per_chunk;
+      j = (j == 0 ? p.n_chunks : j) - 1;
+    }
+  }
+  __device__ __forceinline__ int kv0(const DqParams& p) const { return j * p.chunk_len + tt * 128; }
+  __device__ __forceinline__ int kv_end(const DqParams& p) const { return min(j * p.chunk_len + p.chunk_len, p.L); }
+};
+
+__device__ __forceinline__ void dq_wait_drain(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > ctl.limit_ns) {
+      if (ctl.status) atomicCAS(ctl.status, 0, kErrTimeout | (kQSiteDrain << 8));
+      return;
+    }
+  }
+}
+
+// Dynamic shared memory: 1 KB alignment slack + Q + dO + 3 K slots + 2 V slots + barriers
+// (d = 128: 230,656 bytes).
+__host__ __device__ constexpr size_t bwd_dq_smem_bytes(int d) {
+  return 1024 + static_cast<size_t>(2 + kDqKSlots + kDqVSlots) * 128 * d * 2 + 256;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDqThreads, 1)
+    ring_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const DqParams p) {
+  static_assert(D == 64 || D == 128, "head dim");
+  constexpr int kBoxes = D / 64;
+  constexpr uint32_t kBoxBytes = 128 * 64 * 2;
+  constexpr uint32_t kTile = kBoxes * kBoxBytes;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = smem;
+  uint8_t* do_s = smem + kTile;
+  uint8_t* k_s = smem + 2 * kTile;                  // [kDqKSlots]
+  uint8_t* v_s = k_s + kDqKSlots * kTile;           // [kDqVSlots]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(v_s + kDqVSlots * kTile);
+  // Barriers (a waiter on a two-barrier pair [t & 1] uses parity (t >> 1) & 1; none can run two
+  // phases ahead of its waiter, because each next phase needs that waiter's own progress):
+  //  q_full          Q and dO landed
+  //  k_full[3]       K_i landed in slot i % 3 (parity (i / 3) & 1)
+  //  v_full[2]       V_i landed in slot i % 2 (parity (i / 2) & 1)
+  //  s_full[2]       MMA commit after S(i) (buffer i & 1)
+  //  dp_full[2]      MMA commit after dP(i): dP(i) in TMEM, and V_i no longer read
+  //  dp_free         elementwise -> MMA: dP(i) loaded into registers (4 warp arrivals)
+  //  ds_full[2]      elementwise -> MMA: dS(i) written to TMEM (4 warp arrivals)
+  //  dq_done[2]      MMA commit after dQ += dS(i) K(i): K_i no longer read; after the last
+  //                  tile, dQ is complete
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;                      // [3]
+  uint64_t* v_full = bars + 4;                      // [2]
+  uint64_t* s_full = bars + 6;                      // [2]
+  uint64_t* dp_full = bars + 8;                     // [2]
+  uint64_t* dp_free = bars + 10;
+  uint64_t* ds_full = bars + 11;                    // [2]
+  uint64_t* dq_done = bars + 13;                    // [2]
+  uint64_t* drain_bar = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* skip_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kDqKSlots; ++s) mbar_init(&k_full[s], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&dp_full[s], 1);
+      mbar_init(&ds_full[s], 4);
+      mbar_init(&dq_done[s], 1);
+    }
+    mbar_init(dp_free, 4);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *skip_flag = (p.status != nullptr && *reinterpret_cast<volatile int*>(p.status) != 0) ? 1 : 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (*skip_flag) return;
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const DqItem it = decode_dq_item(p);
+  const int T = it.n_tiles;
+  const uint32_t tDQ = tmem_base, tS0 = tmem_base + 128, tDP = tmem_base + 384;
+
+  if (warp == kDqLoadWarp) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      const uint64_t pol_kv = policy_evict_last();
+      const uint64_t pol_q = policy_evict_first();
+      mbar_arrive_expect_tx(q_full, 2 * kTile);
+#pragma unroll
+      for (int x = 0; x < kBoxes; ++x) {
+        tma_load_4d(q_s + x * kBoxBytes, &tm_q, q_full, x * 64, it.row0, it.h, it.b, pol_q);
+        tma_load_4d(do_s + x * kBoxBytes, &tm_do, q_full, x * 64, it.row0, it.h, it.b, pol_q);
+      }
+      int nk = 0, nv = 0;  // loads issued
+      DqKvIter kvi(p, it);
+      for (int i = 0; i < T; ++i, kvi.next(p)) {
+        const int kv0 = kvi.kv0(p);
+        // K_i takes the slot of K_{i-3}: free once dQ(i-3) completed
+        if (i >= kDqKSlots && !wait_bounded(&dq_done[(i - 3) & 1], ((i - 3) >> 1) & 1, ctl, kQSiteLoadK)) break;
+        {
+          uint64_t* full = &k_full[i % kDqKSlots];
+          uint8_t* dst = k_s + (i % kDqKSlots) * kTile;
+          mbar_arrive_expect_tx(full, kTile);
+#pragma unroll
+          for (int x = 0; x < kBoxes; ++x) tma_load_4d(dst + x * kBoxBytes, &tm_k, full, x * 64, kv0, it.g, it.b, pol_kv);
+          ++nk;
+        }
+        // V_i takes the slot of V_{i-2}: free once dP(i-2) completed
+        if (i >= kDqVSlots && !wait_bounded(&dp_full[(i - 2) & 1], ((i - 2) >> 1) & 1, ctl, kQSiteLoadV)) break;
+        {
+          uint64_t* full = &v_full[i & 1];
+          uint8_t* dst = v_s + (i & 1) * kTile;
+          mbar_arrive_expect_tx(full, kTile);
+#pragma unroll
+          for (int x = 0; x < kBoxes; ++x) tma_load_4d(dst + x * kBoxBytes, &tm_v, full, x * 64, kv0, it.g, it.b, pol_kv);
+          ++nv;
+        }
+      }
+      // drain: every load this thread issued has landed before the CTA can exit
+      dq_wait_drain(q_full, 0, ctl);
+      for (int n = (nk > kDqKSlots ? nk - kDqKSlots : 0); n < nk; ++n)
+        dq_wait_drain(&k_full[n % kDqKSlots], (n / kDqKSlots) & 1, ctl);
+      for (int n = (nv > kDqVSlots ? nv - kDqVSlots : 0); n < nv; ++n) dq_wait_drain(&v_full[n & 1], (n >> 1) & 1, ctl);
+    }
+    __syncwarp();
+  } else if (warp == kDqMmaWarp) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_kk = make_idesc_bf16(128, 128, false);  // S, dP: A and B K-major
+      constexpr uint32_t idesc_o = make_idesc_bf16(128, D, true);      // dQ: A TMEM, B (K) N-major
+      const uint32_t q_a = smem_u32(q_s), do_a = smem_u32(do_s), k_a0 = smem_u32(k_s), v_a0 = smem_u32(v_s);
+      // X = A B^T over d (both tiles d-contiguous), 128 x 128 into TMEM column d_tmem
+      auto issue_kk = [=](uint32_t d_tmem, uint32_t a, uint32_t b) {
+#pragma unroll 1
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          umma_ss(d_tmem, make_sdesc(a + off, 16, 1024), make_sdesc(b + off, 16, 1024), idesc_kk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto wait_k = [&](int i) { return wait_bounded(&k_full[i % kDqKSlots], (i / kDqKSlots) & 1, ctl, kQSiteMmaK); };
+      auto wait_v = [&](int i) { return wait_bounded(&v_full[i & 1], (i >> 1) & 1, ctl, kQSiteMmaV); };
+      auto kaddr = [&](int i) { return k_a0 + (i % kDqKSlots) * kTile; };
+      auto vaddr = [&](int i) { return v_a0 + (i & 1) * kTile; };
+
+      bool ok = wait_bounded(q_full, 0, ctl, kQSiteMmaQ);
+      if (ok && T > 0) {
+        ok = wait_k(0);
+        if (ok) {
+          issue_kk(tS0, q_a, kaddr(0));
+          umma_commit(&s_full[0]);
+          ok = wait_v(0);
+        }
+        if (ok) {
+          issue_kk(tDP, do_a, vaddr(0));
+          umma_commit(&dp_full[0]);
+        }
+      }
+      for (int i = 0; i < T && ok; ++i) {
+        if (i + 1 < T) {
+          // S(i+1) into buffer (i+1)&1, which held dS(i-1): dQ(i-1) was issued before
+          if (!wait_k(i + 1)) { ok = false; break; }
+          issue_kk(tS0 + ((i + 1) & 1) * 128, q_a, kaddr(i + 1));
+          umma_commit(&s_full[(i + 1) & 1]);
+          // dP(i+1) over dP(i), once the elementwise warps hold dP(i) in registers
+          if (!wait_v(i + 1)) { ok = false; break; }
+          if (!wait_bounded(dp_free, i & 1, ctl, kQSiteMmaDpFree)) { ok = false; break; }
+          tc_fence_after();
+          issue_kk(tDP, do_a, vaddr(i + 1));
+          umma_commit(&dp_full[(i + 1) & 1]);
+        }
+        // dQ += dS(i) K(i): A = dS from TMEM (8 columns per 16 keys), B = K N-major
+        if (!wait_bounded(&ds_full[i & 1], (i >> 1) & 1, ctl, kQSiteMmaDs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ds_t = tS0 + (i & 1) * 128;
+        const uint32_t ka = kaddr(i);
+#pragma unroll 1
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tDQ, ds_t + kk * 8, make_sdesc(ka + kk * 2048, kBoxBytes, 1024), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&dq_done[i & 1]);
+      }
+      // drain: all MMAs issued by this thread are complete before TMEM is freed
+      umma_commit(drain_bar);
+      dq_wait_drain(drain_bar, 0, ctl);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ---------------- elementwise (thread = query row) and the dQ epilogue ----------------
+    const uint32_t lofs = (warp * 32u) << 16;
+    const int q_row = it.row0 + static_cast<int>(warp * 32 + lane);
+    const bool q_live = q_row < it.q_end;
+    // rows past the chunk (ragged tail) get LSE = +inf: probability 0, no contribution
+    float lse2 = INFINITY, Dr = 0.f;
+    if (q_live) {
+      lse2 = p.lse[it.b * p.lse_sb + it.h * p.lse_sh + static_cast<long long>(q_row) * p.lse_sl] *
+             1.4426950408889634f;
+      Dr = p.Dvec[(static_cast<long long>(it.b) * p.Hq + it.h) * p.L + q_row];
+    }
+    const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    const uint64_t nl2 = f2_pack(-lse2, -lse2);
+    const uint64_t nD2 = f2_pack(-Dr, -Dr);
+    bool ok = true;
+    DqKvIter kvi(p, it);
+    for (int i = 0; i < T; ++i, kvi.next(p)) {
+      const uint32_t tS = tS0 + (i & 1) * 128 + lofs;
+      const int kv0 = kvi.kv0(p);
+      int lim = kvi.kv_end(p) - kv0;
+      if (p.causal) lim = min(lim, q_row - kv0 + 1);
+      const bool masked = __any_sync(0xffffffffu, lim < 128);
+      if (!__all_sync(0xffffffffu, wait_bounded(&s_full[i & 1], (i >> 1) & 1, ctl, kQSiteS))) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sa[32], sb[32];
+      tmem_ld32(tS + 0, sa);
+      tmem_ld32(tS + 32, sb);
+      if (!__all_sync(0xffffffffu, wait_bounded(&dp_full[i & 1], (i >> 1) & 1, ctl, kQSiteDp))) { ok = false; break; }
+      tc_fence_after();
+      uint32_t dp[4][32];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tDP + lofs + cc * 32, dp[cc]);
+      tmem_wait_ld();
+      // dP(i) is in registers: the MMA may write dP(i+1)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dp_free);
+      // dS of one 32-column chunk -> 16 packed bf16 columns over S columns already read
+      auto ds_chunk = [&](uint32_t (&r)[32], const uint32_t (&g)[32], int cc) {
+        if (masked) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (cc * 32 + e >= lim) r[e] = __float_as_uint(-INFINITY);
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * e2]), __uint_as_float(r[2 * e2 + 1])), sl2x2, nl2), x0, x1);
+          const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          const uint64_t dd = f2_add(f2_pack(__uint_as_float(g[2 * e2]), __uint_as_float(g[2 * e2 + 1])), nD2);
+          float d0, d1;
+          f2_unpack(f2_mul(pp, dd), d0, d1);
+          pk[e2] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tS + cc * 16, pk);
+      };
+      ds_chunk(sa, dp[0], 0);
+      tmem_ld32(tS + 64, sa);
+      ds_chunk(sb, dp[1], 1);
+      tmem_ld32(tS + 96, sb);
+      tmem_wait_ld();
+      ds_chunk(sa, dp[2], 2);
+      ds_chunk(sb, dp[3], 3);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ds_full[i & 1]);
+    }
+    // epilogue: dQ * scale -> bf16
+    if (ok && T > 0 &&
+        __all_sync(0xffffffffu, wait_bounded(&dq_done[(T - 1) & 1], ((T - 1) >> 1) & 1, ctl, kQSiteDone))) {
+      tc_fence_after();
+      __nv_bfloat16* dst = p.dq + it.b * p.dq_sb + it.h * p.dq_sh + static_cast<long long>(q_row) * p.dq_sl;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tDQ + lofs + cc * 32, r);
+        tmem_wait_ld();
+        if (q_live) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v4;
+            v4.x = pack_bf16x2(__uint_as_float(r[e]) * p.scale, __uint_as_float(r[e + 1]) * p.scale);
+            v4.y = pack_bf16x2(__uint_as_float(r[e + 2]) * p.scale, __uint_as_float(r[e + 3]) * p.scale);
+            v4.z = pack_bf16x2(__uint_as_float(r[e + 4]) * p.scale, __uint_as_float(r[e + 5]) * p.scale);
+            v4.w = pack_bf16x2(__uint_as_float(r[e + 6]) * p.scale, __uint_as_float(r[e + 7]) * p.scale);
+            *reinterpret_cast<uint4*>(dst + cc * 32 + e) = v4;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace cpattn

@@ -5,30 +5,30 @@
 // group:  P = exp(scale S - LSE);  dV += P^T dO;  dP = dO V^T;  dS = P o (dP - D) with
 // D = rowsum(dO o O);  dQ += scale dS K;  dK += scale dS^T Q.
 //
+// The backward runs as two kernels with no atomics: this one (key-stationary) computes dK and
+// dV, bwd_dq_kernel.cuh (query-stationary) computes dQ; each recomputes S and dP for itself.
+//
 // Ring order: the CTA owns one 128-row KV tile of chunk j and visits the query chunks of the
 // ranks that see it — r = j (the diagonal chunk, masked key <= query), j+1, ..., N-1 — and,
 // for each 128-row query tile, every query head of the KV group.  dK and dV accumulate in
-// TMEM over the whole visit (the sum over the group's heads happens there, without atomics);
-// dQ is added into an fp32 accumulator in global memory.
+// TMEM over the whole visit (the sum over the group's heads happens there, without atomics).
 //
-// Warp roles (320 threads):
+// Warp roles (192 threads):
 //   warps 0-3  P / dS warps: thread t <-> key row t <-> TMEM lane t; epilogue writes dK, dV
-//   warps 4-7  dQ warps: thread t <-> query row t of the dQ tile; float4 atomics into dQ_acc
-//   warp  8    loads: K, V once (TMA); per query tile Q_i, dO_i (TMA, 2 stages) and
+//   warp  4    loads: K, V once (TMA); per query tile Q_i, dO_i (TMA, 2 stages) and
 //              LSE_i, D_i (plain loads into shared memory)
-//   warp  9    MMA issuer (one thread)
-// TMEM columns: S^T/P^T [0,128)  dP^T/dS^T, then dQ [128,256)  dV [256,384)  dK [384,512).
+//   warp  5    MMA issuer (one thread)
+// TMEM columns: S^T/P^T [0,128)  dP^T/dS^T [128,256)  dV [256,384)  dK [384,512).
 #pragma once
 #include <cstddef>
 #include "sm100.cuh"
 
 namespace cpattn {
 
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 192;
+constexpr int kBwdLoadWarp = 4;
+constexpr int kBwdMmaWarp = 5;
 constexpr uint32_t kBwdTmemCols = 512;
-
-// Extra workspace the backward kernels need beyond the dQ accumulator and D.
-inline size_t bwd_workspace_extra(int, int, int, int, int) { return 0; }
 
 enum BwdSite : int {
   kBSiteLoadEmpty = 17, kBSiteMmaKV = 18, kBSiteMmaQ = 19, kBSiteMmaDq = 20, kBSiteMmaP = 21,
@@ -44,7 +44,6 @@ struct BwdParams {
   const float* lse;   // [B, Hq, L] natural-log LSE of the forward
   long long lse_sb, lse_sh, lse_sl;
   const float* Dvec;  // [B, Hq, L] rowsum(dO * O), contiguous
-  float* dq_acc;      // [B, Hq, L, d] fp32, contiguous, zeroed before the launch
   __nv_bfloat16* dk;  // [B, Hkv, L, d]
   long long dk_sb, dk_sh, dk_sl;
   __nv_bfloat16* dv;
@@ -120,11 +119,9 @@ __device__ __forceinline__ void bwd_wait_drain(uint64_t* bar, uint32_t parity, c
   }
 }
 
-// Shared memory (d = 128): K 32K | V 32K | Q[2] 64K | dO[2] 64K | dS 32K | LSE/D[2] 2K | barriers.
-// The dS tile is 128 keys x 128 queries whatever d is.
-constexpr size_t kBwdDsBytes = 128 * 128 * 2;
+// Shared memory (d = 128): K 32K | V 32K | Q[2] 64K | dO[2] 64K | LSE/D[2] 2K | barriers.
 __host__ __device__ constexpr size_t bwd_smem_bytes(int d) {
-  return static_cast<size_t>(6) * 128 * d * 2 + kBwdDsBytes + 2 * 1024 + 256;
+  return static_cast<size_t>(6) * 128 * d * 2 + 2 * 1024 + 256;
 }
 
 template <int D>
@@ -140,9 +137,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* v_s = smem + kTile;
   uint8_t* q_s = smem + 2 * kTile;    // [2]
   uint8_t* do_s = smem + 4 * kTile;   // [2]
-  uint8_t* ds_s = smem + 6 * kTile;   // dS, query-major halves of 64 queries (16 KB each)
-  float* stat_s = reinterpret_cast<float*>(smem + 6 * kTile + kBwdDsBytes);  // [2][256]: lse2, D
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * kTile + kBwdDsBytes + 2048);
+  float* stat_s = reinterpret_cast<float*>(smem + 6 * kTile);  // [2][256]: lse2, D
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * kTile + 2048);
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;     // [2]
   uint64_t* q_empty = bars + 3;    // [2]
@@ -150,8 +146,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* dp_full = bars + 6;
   uint64_t* p_full = bars + 7;
   uint64_t* ds_full = bars + 8;
-  uint64_t* dq_full = bars + 9;
-  uint64_t* dq_free = bars + 10;
   uint64_t* done_bar = bars + 11;
   uint64_t* drain_bar = bars + 12;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
@@ -172,8 +166,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(dp_full, 1);
     mbar_init(p_full, 4);
     mbar_init(ds_full, 4);
-    mbar_init(dq_full, 1);
-    mbar_init(dq_free, 4);
     mbar_init(done_bar, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -197,7 +189,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const BwdItem it = decode_bwd_item(p);
   const uint32_t tS = tmem_base, tDP = tmem_base + 128, tDV = tmem_base + 256, tDK = tmem_base + 384;
 
-  if (warp == 8) {
+  if (warp == kBwdLoadWarp) {
     // ---------------- loads ----------------
     const uint64_t pol_keep = policy_evict_last();
     if (lane == 0) {
@@ -254,13 +246,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int s2 = (issued > 2 ? issued - 2 : 0); s2 < issued; ++s2) bwd_wait_drain(&q_full[s2 & 1], (s2 >> 1) & 1, ctl);
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == kBwdMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_kk = make_idesc_bf16(128, 128, false);     // S^T, dP^T: both K-major
       constexpr uint32_t idesc_tn = make_idesc_bf16(128, D, true);        // dV, dK: A TMEM, B N-major
-      constexpr uint32_t idesc_nn = make_idesc_bf16(128, D, true) | (1u << 15);  // dQ: A, B N-major
-      const uint32_t k_a = smem_u32(k_s), v_a = smem_u32(v_s), ds_a = smem_u32(ds_s);
+      const uint32_t k_a = smem_u32(k_s), v_a = smem_u32(v_s);
       bool ok = wait_bounded(kv_full, 0, ctl, kBSiteMmaKV);
       for (int i = 0; i < it.n_iter && ok; ++i) {
         const int st = i & 1;
@@ -274,9 +265,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           umma_ss(tS, make_sdesc(k_a + off, 16, 1024), make_sdesc(q_a + off, 16, 1024), idesc_kk, kk > 0);
         }
         umma_commit(s_full);
-        // (2) dP^T = V dO^T, into the columns that held dQ of the previous tile
-        if (i > 0 && !wait_bounded(dq_free, (i - 1) & 1, ctl, kBSiteMmaDq)) { ok = false; break; }
-        tc_fence_after();
+        // (2) dP^T = V dO^T, over dS^T of the previous tile (its dK MMA was issued before)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
@@ -295,12 +284,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
           umma_ts(tDK, tDP + kk * 8, make_sdesc(q_a + kk * 2048, kBoxBytes, 1024), idesc_tn, (i > 0 || kk > 0));
-        // (5) dQ_i = dS K  [A = dS query-major in smem, B = K N-major], over dP^T/dS^T
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ss(tDP, make_sdesc(ds_a + kk * 2048, kBoxBytes, 1024), make_sdesc(k_a + kk * 2048, kBoxBytes, 1024),
-                  idesc_nn, kk > 0);
-        umma_commit(dq_full);
         umma_commit(&q_empty[st]);
       }
       if (ok) umma_commit(done_bar);
@@ -369,18 +352,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           dsk[e >> 1] = pack_bf16x2(d0, d1);
         }
         tmem_st16(tDP + lofs + cc * 16, dsk);
-        // dS for the dQ MMA: query-major, two 64-query halves of [128 keys x 128 B], 128-byte
-        // swizzle (16-byte chunk index XOR key row % 8); this chunk = queries [32cc, 32cc+32)
-        uint8_t* half = ds_s + (cc >> 1) * kBoxBytes + t * 128;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int chunk = (cc & 1) * 4 + u;
-          *reinterpret_cast<uint4*>(half + ((chunk ^ (t & 7)) << 4)) =
-              make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]);
-        }
       }
       tmem_wait_st();
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_full);
@@ -418,35 +391,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
       }
-    }
-  } else {
-    // ---------------- dQ (warps 4-7, thread = query row of the tile) ----------------
-    const uint32_t lane_base = (warp & 3) * 32;
-    const int t = lane_base + lane;
-    const uint32_t lofs = lane_base << 16;
-    for (int i = 0; i < it.n_iter; ++i) {
-      int h, q0, q_end;
-      bwd_qtile(p, it, i, h, q0, q_end);
-      const int q = q0 + t;
-      if (!__all_sync(0xffffffffu, wait_bounded(dq_full, i & 1, ctl, kBSiteDqFull))) break;
-      tc_fence_after();
-      float* dst = p.dq_acc + ((static_cast<long long>(it.b) * p.Hq + h) * p.L + q) * D;
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tDP + lofs + cc * 32, r);
-        tmem_wait_ld();
-        if (q < q_end) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            atomicAdd(reinterpret_cast<float4*>(dst + cc * 32 + e),
-                      make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
-                                  __uint_as_float(r[e + 3])));
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dq_free);
     }
   }
 

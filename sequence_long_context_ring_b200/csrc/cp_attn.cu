@@ -12,6 +12,7 @@
 #include <new>
 
 #include "aux_kernels.cuh"
+#include "bwd_dq_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "fwd_kernel.cuh"
 
@@ -252,6 +253,17 @@ cp_status_t launch_bwd_d(const BwdParams& p, const CUtensorMap& mq, const CUtens
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
+template <int D>
+cp_status_t launch_bwd_dq_d(const DqParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const CUtensorMap& mdo, int64_t grid, cudaStream_t s) {
+  const size_t smem = bwd_dq_smem_bytes(D);
+  if (cudaFuncSetAttribute(ring_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return CP_ERR_CUDA;
+  ring_bwd_dq_kernel<D><<<(unsigned)grid, kDqThreads, smem, s>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
 // D = rowsum(dO * O) for [b, h, l] rows given by per-axis element strides.
 cp_status_t launch_rowdot(const void* o, const int64_t os[3], const void* g, const int64_t gs[3], float* D, int B,
                           int H, int L, int d, cudaStream_t s) {
@@ -260,15 +272,6 @@ cp_status_t launch_rowdot(const void* o, const int64_t os[3], const void* g, con
   const int64_t threads = (int64_t)B * H * L * (d / 8);
   if (threads == 0) return CP_OK;
   rowdot_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
-}
-
-cp_status_t launch_cast(const float* src, __nv_bfloat16* dst, float scale, int B, int H, int L, int d, int64_t sb,
-                        int64_t sh, int64_t sl, cudaStream_t s) {
-  CastParams p{src, dst, scale, B, H, L, d, sb, sh, sl};
-  const int64_t n4 = (int64_t)B * H * L * d / 4;
-  if (n4 == 0) return CP_OK;
-  cast_bf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
@@ -310,8 +313,6 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
   const size_t nq = (size_t)c.B * c.Hq * c.L * c.d, nkv = (size_t)c.B * c.Hkv * c.L * c.d;
   const size_t nrow = (size_t)c.B * c.Hq * c.L;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  float* dq_acc = reinterpret_cast<float*>(w);
-  w += align256(nq * 4);
   float* Dvec = reinterpret_cast<float*>(w);
   w += align256(nrow * 4);
 
@@ -320,10 +321,9 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
   const int64_t gs[3] = {dout->stride[0], seq ? dout->stride[2] : dout->stride[1],
                          seq ? dout->stride[1] : dout->stride[2]};
   CP_TRY(launch_rowdot(o->data, os, dout->data, gs, Dvec, c.B, c.Hq, c.L, c.d, s));
-  if (cudaMemsetAsync(dq_acc, 0, nq * 4, s) != cudaSuccess) return CP_ERR_CUDA;
 
   View vq, vk, vv, vdo;
-  void *dqh = nullptr, *dkh = nullptr, *dvh = nullptr;
+  void *dkh = nullptr, *dvh = nullptr;
   if (!seq) {
     vq = view_of(q);
     vk = view_of(k);
@@ -333,8 +333,6 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
     void* qh = w;
     w += align256(nq * 2);
     void* doh = w;
-    w += align256(nq * 2);
-    dqh = w;
     w += align256(nq * 2);
     void* kh = w;
     w += align256(nkv * 2);
@@ -373,7 +371,6 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
   p.lse_sh = lse->stride[1];
   p.lse_sl = lse->stride[2];
   p.Dvec = Dvec;
-  p.dq_acc = dq_acc;
   if (!seq) {
     p.dk = static_cast<__nv_bfloat16*>(dk->data);
     p.dk_sb = dk->stride[0];
@@ -403,14 +400,40 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
   } else {
     CP_TRY(launch_bwd_d<64>(p, mq, mk, mv, mdo, grid, s));
   }
-  if (!seq) {
-    return launch_cast(dq_acc, static_cast<__nv_bfloat16*>(dq->data), plan->scale, c.B, c.Hq, c.L, c.d,
-                       dq->stride[0], dq->stride[1], dq->stride[2], s);
+  // dQ, query-stationary: written once, scaled, as bf16 straight into dq (in the caller's
+  // layout: [b, h, l] strides of either the head-major or the sequence-major tensor)
+  DqParams qp{};
+  qp.B = c.B;
+  qp.Hq = c.Hq;
+  qp.Hkv = c.Hkv;
+  qp.L = c.L;
+  qp.d = c.d;
+  qp.G = plan->G;
+  qp.n_chunks = p.n_chunks;
+  qp.chunk_len = p.chunk_len;
+  qp.tiles_per_chunk = p.tiles_per_chunk;
+  qp.causal = p.causal;
+  qp.scale = p.scale;
+  qp.scale_log2 = p.scale_log2;
+  qp.lse = p.lse;
+  qp.lse_sb = p.lse_sb;
+  qp.lse_sh = p.lse_sh;
+  qp.lse_sl = p.lse_sl;
+  qp.Dvec = Dvec;
+  qp.dq = static_cast<__nv_bfloat16*>(dq->data);
+  qp.dq_sb = dq->stride[0];
+  qp.dq_sh = seq ? dq->stride[2] : dq->stride[1];
+  qp.dq_sl = seq ? dq->stride[1] : dq->stride[2];
+  qp.status = sw;
+  qp.wait_limit_ns = p.wait_limit_ns;
+  const int64_t qgrid = (int64_t)qp.n_chunks * qp.tiles_per_chunk * c.B * c.Hq;
+  if (c.d == 128) {
+    CP_TRY(launch_bwd_dq_d<128>(qp, mq, mk, mv, mdo, qgrid, s));
+  } else {
+    CP_TRY(launch_bwd_dq_d<64>(qp, mq, mk, mv, mdo, qgrid, s));
   }
-  CP_TRY(launch_cast(dq_acc, static_cast<__nv_bfloat16*>(dqh), plan->scale, c.B, c.Hq, c.L, c.d,
-                     (int64_t)c.Hq * c.L * c.d, (int64_t)c.L * c.d, c.d, s));
-  // all-to-all head -> seq of the gradients
-  CP_TRY(head_buf_to_seq(dqh, dq, s));
+  if (!seq) return CP_OK;
+  // all-to-all head -> seq of dK and dV
   CP_TRY(head_buf_to_seq(dkh, dk, s));
   return head_buf_to_seq(dvh, dv, s);
 }
@@ -491,8 +514,8 @@ cp_status_t cp_attn_workspace_size(const cp_plan_t* plan, int backward, size_t* 
   if (!backward) {
     if (seq_major) ws = 2 * align256(nq * 2) + 2 * align256(nkv * 2);
   } else {
-    ws = align256(nq * 4) + align256(nrow * 4) + bwd_workspace_extra(c.B, c.Hq, c.Hkv, c.L, c.d);
-    if (seq_major) ws += 3 * align256(nq * 2) + 4 * align256(nkv * 2);  // q, do, dq ; k, v, dk, dv
+    ws = align256(nrow * 4);                                             // D
+    if (seq_major) ws += 2 * align256(nq * 2) + 4 * align256(nkv * 2);  // q, do ; k, v, dk, dv
   }
   *bytes = ws;
   return CP_OK;

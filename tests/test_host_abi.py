@@ -94,4 +94,8 @@ def test_workspace_sizes():
     assert p.workspace_size(False) >= 4 * 32 * 131072 * 128 * 2
     r = Plan(B=1, Hq=4, Hkv=4, L=1024, d=64, n_cp=4)
     assert r.workspace_size(False) == 0
-    assert r.workspace_size(True) >= 4 * 1024 * 64 * 4
+    # ring backward: only D = rowsum(dO * O), fp32 [B, Hq, L] (dQ has no accumulator)
+    assert r.workspace_size(True) == 4 * 1024 * 4
+    # sequence-major backward: D plus head-major copies of q, dO (Hq) and k, v, dk, dv (Hkv)
+    n = 32 * 131072 * 128 * 2
+    assert p.workspace_size(True) == 32 * 131072 * 4 + 2 * n + 4 * n
