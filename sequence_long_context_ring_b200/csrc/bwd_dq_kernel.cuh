@@ -8,12 +8,16 @@
 // dQ accumulates in TMEM over the whole visit and is written once, scaled and rounded to
 // bf16: no atomics, and the result does not depend on the order in which CTAs run.
 //
-// Warp roles (192 threads):
-//   warps 0-3  elementwise: thread t <-> query row t <-> TMEM lane t; epilogue writes dQ
-//   warp  4    loads: Q and dO once; K_i into a 3-slot ring, V_i into a 2-slot ring (TMA)
-//   warp  5    MMA issuer (one thread)
+// Warp roles (320 threads):
+//   warps 0-7  elementwise: warp w handles query rows 32(w%4) .. +31 (thread <-> TMEM lane)
+//              and keys [64(w/4), 64(w/4) + 64) -- no row reduction is needed (LSE and D are
+//              known), so the two warpgroups split the columns; epilogue writes dQ (each
+//              warpgroup half of the d columns)
+//   warp  8    loads: Q and dO once; K_i into a 3-slot ring, V_i into a 2-slot ring (TMA)
+//   warp  9    MMA issuer (one thread)
 // TMEM columns: dQ [0,128)  S buffer 0 [128,256)  S buffer 1 [256,384)  dP [384,512).
-// S(i) goes to buffer i&1; dS(i) (bf16, two per column) overwrites the first 64 columns of it.
+// S(i) goes to buffer i&1; dS(i) of keys [64h, 64h+64) (bf16, two per column) overwrites
+// columns [64h, 64h+32) of it, which warpgroup h has already read.
 // Per iteration the MMA issues S(i+1) and dP(i+1) before dQ += dS(i) K(i), so the tensor pipe
 // computes the next tile's products while the elementwise warps work on this one.
 #pragma once
@@ -21,9 +25,9 @@
 
 namespace cpattn {
 
-constexpr int kDqThreads = 192;
-constexpr int kDqLoadWarp = 4;
-constexpr int kDqMmaWarp = 5;
+constexpr int kDqThreads = 320;
+constexpr int kDqLoadWarp = 8;
+constexpr int kDqMmaWarp = 9;
 constexpr int kDqKSlots = 3;
 constexpr int kDqVSlots = 2;
 
@@ -127,8 +131,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   //  v_full[2]       V_i landed in slot i % 2 (parity (i / 2) & 1)
   //  s_full[2]       MMA commit after S(i) (buffer i & 1)
   //  dp_full[2]      MMA commit after dP(i): dP(i) in TMEM, and V_i no longer read
-  //  dp_free         elementwise -> MMA: dP(i) loaded into registers (4 warp arrivals)
-  //  ds_full[2]      elementwise -> MMA: dS(i) written to TMEM (4 warp arrivals)
+  //  dp_free         elementwise -> MMA: dP(i) loaded into registers (8 warp arrivals)
+  //  ds_full[2]      elementwise -> MMA: dS(i) written to TMEM (8 warp arrivals)
   //  dq_done[2]      MMA commit after dQ += dS(i) K(i): K_i no longer read; after the last
   //                  tile, dQ is complete
   uint64_t* q_full = bars + 0;
@@ -155,10 +159,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&dp_full[s], 1);
-      mbar_init(&ds_full[s], 4);
+      mbar_init(&ds_full[s], 8);
       mbar_init(&dq_done[s], 1);
     }
-    mbar_init(dp_free, 4);
+    mbar_init(dp_free, 8);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     *skip_flag = (p.status != nullptr && *reinterpret_cast<volatile int*>(p.status) != 0) ? 1 : 0;
@@ -276,8 +280,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const uint32_t ds_t = tS0 + (i & 1) * 128;
         const uint32_t ka = kaddr(i);
 #pragma unroll 1
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tDQ, ds_t + kk * 8, make_sdesc(ka + kk * 2048, kBoxBytes, 1024), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)  // keys [16 kk, 16 kk + 16): written by warpgroup kk / 4
+          umma_ts(tDQ, ds_t + 64u * (kk >> 2) + 8u * (kk & 3), make_sdesc(ka + kk * 2048, kBoxBytes, 1024), idesc_o,
+                  (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&dq_done[i & 1]);
       }
       // drain: all MMAs issued by this thread are complete before TMEM is freed
@@ -285,10 +290,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       dq_wait_drain(drain_bar, 0, ctl);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ---------------- elementwise (thread = query row) and the dQ epilogue ----------------
-    const uint32_t lofs = (warp * 32u) << 16;
-    const int q_row = it.row0 + static_cast<int>(warp * 32 + lane);
+  } else if (warp < 8) {
+    // ---------------- elementwise (thread = query row, 64 keys) and the dQ epilogue ----------
+    const uint32_t quarter = warp & 3;
+    const int hh = static_cast<int>(warp >> 2);  // key half
+    const uint32_t lofs = (quarter * 32u) << 16;
+    const int q_row = it.row0 + static_cast<int>(quarter * 32 + lane);
     const bool q_live = q_row < it.q_end;
     // rows past the chunk (ragged tail) get LSE = +inf: probability 0, no contribution
     float lse2 = INFINITY, Dr = 0.f;
@@ -304,11 +311,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     bool ok = true;
     DqKvIter kvi(p, it);
     for (int i = 0; i < T; ++i, kvi.next(p)) {
-      const uint32_t tS = tS0 + (i & 1) * 128 + lofs;
-      const int kv0 = kvi.kv0(p);
+      const uint32_t tS = tS0 + (i & 1) * 128 + lofs + hh * 64;
+      const int kv0 = kvi.kv0(p) + hh * 64;  // first key of this warp's half
       int lim = kvi.kv_end(p) - kv0;
       if (p.causal) lim = min(lim, q_row - kv0 + 1);
-      const bool masked = __any_sync(0xffffffffu, lim < 128);
+      const bool masked = __any_sync(0xffffffffu, lim < 64);
       if (!__all_sync(0xffffffffu, wait_bounded(&s_full[i & 1], (i >> 1) & 1, ctl, kQSiteS))) { ok = false; break; }
       tc_fence_after();
       uint32_t sa[32], sb[32];
@@ -316,15 +323,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       tmem_ld32(tS + 32, sb);
       if (!__all_sync(0xffffffffu, wait_bounded(&dp_full[i & 1], (i >> 1) & 1, ctl, kQSiteDp))) { ok = false; break; }
       tc_fence_after();
-      uint32_t dp[4][32];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tDP + lofs + cc * 32, dp[cc]);
+      uint32_t dpa[32], dpb[32];
+      tmem_ld32(tDP + lofs + hh * 64, dpa);
+      tmem_ld32(tDP + lofs + hh * 64 + 32, dpb);
       tmem_wait_ld();
       // dP(i) is in registers: the MMA may write dP(i+1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dp_free);
-      // dS of one 32-column chunk -> 16 packed bf16 columns over S columns already read
+      // dS of one 32-key chunk -> 16 packed bf16 columns
       auto ds_chunk = [&](uint32_t (&r)[32], const uint32_t (&g)[32], int cc) {
         if (masked) {
 #pragma unroll
@@ -344,25 +351,21 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         tmem_st16(tS + cc * 16, pk);
       };
-      ds_chunk(sa, dp[0], 0);
-      tmem_ld32(tS + 64, sa);
-      ds_chunk(sb, dp[1], 1);
-      tmem_ld32(tS + 96, sb);
-      tmem_wait_ld();
-      ds_chunk(sa, dp[2], 2);
-      ds_chunk(sb, dp[3], 3);
+      ds_chunk(sa, dpa, 0);
+      ds_chunk(sb, dpb, 1);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_full[i & 1]);
     }
-    // epilogue: dQ * scale -> bf16
+    // epilogue: dQ * scale -> bf16, d columns of this warpgroup's half
     if (ok && T > 0 &&
         __all_sync(0xffffffffu, wait_bounded(&dq_done[(T - 1) & 1], ((T - 1) >> 1) & 1, ctl, kQSiteDone))) {
       tc_fence_after();
       __nv_bfloat16* dst = p.dq + it.b * p.dq_sb + it.h * p.dq_sh + static_cast<long long>(q_row) * p.dq_sl;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int c2 = 0; c2 < D / 64; ++c2) {
+        const int cc = hh * (D / 64) + c2;
         uint32_t r[32];
         tmem_ld32(tDQ + lofs + cc * 32, r);
         tmem_wait_ld();

@@ -13,21 +13,30 @@
 // for each 128-row query tile, every query head of the KV group.  dK and dV accumulate in
 // TMEM over the whole visit (the sum over the group's heads happens there, without atomics).
 //
-// Warp roles (192 threads):
-//   warps 0-3  P / dS warps: thread t <-> key row t <-> TMEM lane t; epilogue writes dK, dV
-//   warp  4    loads: K, V once (TMA); per query tile Q_i, dO_i (TMA, 2 stages) and
+// Warp roles (320 threads):
+//   warps 0-7  P / dS warps: warp w handles key rows 32(w%4) .. +31 (thread <-> TMEM lane)
+//              and query columns [64(w/4), 64(w/4) + 64) of S^T and dP^T -- the elementwise
+//              work has no row reduction (LSE and D are known), so it splits by columns;
+//              the epilogue writes dK, dV (each warpgroup half of the d columns)
+//   warp  8    loads: K, V once (TMA); per query tile Q_i, dO_i (TMA, 2 stages) and
 //              LSE_i, D_i (plain loads into shared memory)
-//   warp  5    MMA issuer (one thread)
-// TMEM columns: S^T/P^T [0,128)  dP^T/dS^T [128,256)  dV [256,384)  dK [384,512).
+//   warp  9    MMA issuer (one thread)
+// TMEM columns: S^T [0,128)  dP^T [128,256)  dV [256,384)  dK [384,512).  P^T (bf16, two per
+// column) of query columns [64h, 64h+64) is written over S^T columns [64h, 64h+32), which
+// that warpgroup has already read; dS^T likewise over dP^T.
 #pragma once
 #include <cstddef>
 #include "sm100.cuh"
 
 namespace cpattn {
 
-constexpr int kBwdThreads = 192;
-constexpr int kBwdLoadWarp = 4;
-constexpr int kBwdMmaWarp = 5;
+constexpr int kBwdThreads = 320;
+constexpr int kBwdLoadWarp = 8;
+constexpr int kBwdMmaWarp = 9;
+
+// TMEM column (inside S^T or dP^T) of the bf16 A operand for queries [16 kk, 16 kk + 16):
+// warpgroup kk/4 wrote them at the start of its own column half.
+__device__ __forceinline__ uint32_t bwd_a_col(int kk) { return 64u * (kk >> 2) + 8u * (kk & 3); }
 constexpr uint32_t kBwdTmemCols = 512;
 
 enum BwdSite : int {
@@ -164,8 +173,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(ds_full, 4);
+    mbar_init(p_full, 8);
+    mbar_init(ds_full, 8);
     mbar_init(done_bar, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -277,13 +286,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tDV, tS + kk * 8, make_sdesc(do_a + kk * 2048, kBoxBytes, 1024), idesc_tn, (i > 0 || kk > 0));
+          umma_ts(tDV, tS + bwd_a_col(kk), make_sdesc(do_a + kk * 2048, kBoxBytes, 1024), idesc_tn,
+                  (i > 0 || kk > 0));
         // (4) dK += dS^T Q  [A = dS^T in TMEM, B = Q N-major]
         if (!wait_bounded(ds_full, i & 1, ctl, kBSiteMmaDs)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tDK, tDP + kk * 8, make_sdesc(q_a + kk * 2048, kBoxBytes, 1024), idesc_tn, (i > 0 || kk > 0));
+          umma_ts(tDK, tDP + bwd_a_col(kk), make_sdesc(q_a + kk * 2048, kBoxBytes, 1024), idesc_tn,
+                  (i > 0 || kk > 0));
         umma_commit(&q_empty[st]);
       }
       if (ok) umma_commit(done_bar);
@@ -291,32 +302,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bwd_wait_drain(drain_bar, 0, ctl);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ---------------- P / dS (thread = key row) and the dK / dV epilogue ----------------
-    const uint32_t lane_base = warp * 32;
+  } else if (warp < 8) {
+    // ---------------- P / dS (thread = key row, 64 query columns) and the dK / dV epilogue ----
+    const uint32_t lane_base = (warp & 3) * 32;
+    const int hh = static_cast<int>(warp >> 2);     // query-column half
     const int t = lane_base + lane;
     const int kv_row = it.kv0 + t;
     const bool kv_live = kv_row < it.kv_end;
     const uint32_t lofs = lane_base << 16;
+    const uint32_t tSh = tS + lofs + hh * 64, tDPh = tDP + lofs + hh * 64;
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int i = 0; i < it.n_iter; ++i) {
       const int st = i & 1;
       int h, q0, q_end;
       bwd_qtile(p, it, i, h, q0, q_end);
-      const float* lse2 = stat_s + st * 256;
-      const float* dvec = lse2 + 128;
-      // causal: query columns c < kv_row - q0 do not see this key
-      const int c_lo = p.causal ? (kv_row - q0) : 0;
+      const float* lse2 = stat_s + st * 256 + hh * 64;
+      const float* dvec = stat_s + st * 256 + 128 + hh * 64;
+      // causal: query columns c < kv_row - q0 do not see this key (c relative to this half)
+      const int c_lo = p.causal ? (kv_row - q0 - hh * 64) : 0;
       if (!__all_sync(0xffffffffu, wait_bounded(s_full, i & 1, ctl, kBSiteSoftS))) { ok = false; break; }
       tc_fence_after();
-      uint32_t pk[64];  // P^T row as bf16 pairs, kept for dS
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tS + lofs + cc * 32, r);
-        tmem_wait_ld();
-        uint32_t pst[16];
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tSh, ra);
+      tmem_ld32(tSh + 32, rb);
+      tmem_wait_ld();
+      uint32_t pk[32];  // P^T of the 64 columns as bf16 pairs, kept for dS
+      auto p_chunk = [&](const uint32_t (&r)[32], int cc) {
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int c = cc * 32 + e;
@@ -324,12 +336,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           float p1 = ex2_approx(fmaf(__uint_as_float(r[e + 1]), sl2, -lse2[c + 1]));
           if (!kv_live || c < c_lo) p0 = 0.f;
           if (!kv_live || c + 1 < c_lo) p1 = 0.f;
-          pst[e >> 1] = pack_bf16x2(p0, p1);
-          pk[c >> 1] = pst[e >> 1];
+          pk[c >> 1] = pack_bf16x2(p0, p1);
         }
-        // P^T columns [16cc, 16cc+16) overwrite S^T columns already read (in-place stream)
-        tmem_st16(tS + lofs + cc * 16, pst);
-      }
+      };
+      p_chunk(ra, 0);
+      p_chunk(rb, 1);
+      tmem_st16(tSh, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+      tmem_st16(tSh + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -337,28 +350,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
       if (!__all_sync(0xffffffffu, wait_bounded(dp_full, i & 1, ctl, kBSiteSoftDp))) { ok = false; break; }
       tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tDP + lofs + cc * 32, r);
-        tmem_wait_ld();
-        uint32_t dsk[16];
+      tmem_ld32(tDPh, ra);
+      tmem_ld32(tDPh + 32, rb);
+      tmem_wait_ld();
+      uint32_t dsk[32];
+      auto ds_chunk = [&](const uint32_t (&r)[32], int cc) {
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int c = cc * 32 + e;
           const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[c >> 1]));
           const float d0 = pp.x * (__uint_as_float(r[e]) - dvec[c]);
           const float d1 = pp.y * (__uint_as_float(r[e + 1]) - dvec[c + 1]);
-          dsk[e >> 1] = pack_bf16x2(d0, d1);
+          dsk[c >> 1] = pack_bf16x2(d0, d1);
         }
-        tmem_st16(tDP + lofs + cc * 16, dsk);
-      }
+      };
+      ds_chunk(ra, 0);
+      ds_chunk(rb, 1);
+      tmem_st16(tDPh, *reinterpret_cast<const uint32_t(*)[16]>(dsk));
+      tmem_st16(tDPh + 16, *reinterpret_cast<const uint32_t(*)[16]>(dsk + 16));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_full);
     }
-    // epilogue: dV, dK (scaled) for this thread's key row
+    // epilogue: dV, dK (scaled) for this thread's key row, d columns of this warpgroup's half
     const bool have = it.n_iter > 0;
     if (ok && (!have || __all_sync(0xffffffffu, wait_bounded(done_bar, 0, ctl, kBSiteDone)))) {
       tc_fence_after();
@@ -369,7 +384,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         __nv_bfloat16* dst = which == 0 ? p.dv + it.b * p.dv_sb + it.g * p.dv_sh + static_cast<long long>(kv_row) * p.dv_sl
                                         : p.dk + it.b * p.dk_sb + it.g * p.dk_sh + static_cast<long long>(kv_row) * p.dk_sl;
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
+        for (int c2 = 0; c2 < D / 64; ++c2) {
+          const int cc = hh * (D / 64) + c2;
           uint32_t r[32];
           if (have) {
             tmem_ld32(tsrc + cc * 32, r);
