@@ -28,8 +28,13 @@ namespace cpattn {
 constexpr int kDqThreads = 320;
 constexpr int kDqLoadWarp = 8;
 constexpr int kDqMmaWarp = 9;
-constexpr int kDqKSlots = 3;
-constexpr int kDqVSlots = 2;
+#ifndef CPATTN_DQ_KSLOTS
+#define CPATTN_DQ_KSLOTS 3
+#endif
+// K_i is read by S(i) (issued one iteration early) and by dQ(i): it holds its slot about two
+// iterations, V_i (read by dP(i) only) about one, so K gets more of the five slots.
+constexpr int kDqKSlots = CPATTN_DQ_KSLOTS;
+constexpr int kDqVSlots = 5 - kDqKSlots;
 
 enum DqSite : int {
   kQSiteLoadK = 33, kQSiteLoadV = 34, kQSiteMmaQ = 35, kQSiteMmaK = 36, kQSiteMmaV = 37, kQSiteMmaDpFree = 38,
@@ -127,24 +132,23 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   // Barriers (a waiter on a two-barrier pair [t & 1] uses parity (t >> 1) & 1; none can run two
   // phases ahead of its waiter, because each next phase needs that waiter's own progress):
   //  q_full          Q and dO landed
-  //  k_full[3]       K_i landed in slot i % 3 (parity (i / 3) & 1)
-  //  v_full[2]       V_i landed in slot i % 2 (parity (i / 2) & 1)
+  //  k_full[kK]      K_i landed in slot i % kK (parity (i / kK) & 1)
+  //  v_full[kV]      V_i landed in slot i % kV (parity (i / kV) & 1)
+  //  k_free[kK]      MMA commit after dQ(i): slot i % kK (K_i) no longer read
   //  s_full[2]       MMA commit after S(i) (buffer i & 1)
   //  dp_full[2]      MMA commit after dP(i): dP(i) in TMEM, and V_i no longer read
   //  dp_free         elementwise -> MMA: dP(i) loaded into registers (8 warp arrivals)
   //  ds_full[2]      elementwise -> MMA: dS(i) written to TMEM (8 warp arrivals)
-  //  dq_done[2]      MMA commit after dQ += dS(i) K(i): K_i no longer read; after the last
-  //                  tile, dQ is complete
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;                      // [3]
-  uint64_t* v_full = bars + 4;                      // [2]
-  uint64_t* s_full = bars + 6;                      // [2]
-  uint64_t* dp_full = bars + 8;                     // [2]
-  uint64_t* dp_free = bars + 10;
-  uint64_t* ds_full = bars + 11;                    // [2]
-  uint64_t* dq_done = bars + 13;                    // [2]
-  uint64_t* drain_bar = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* k_full = bars + 1;                      // [kK]
+  uint64_t* v_full = k_full + kDqKSlots;            // [kV]
+  uint64_t* k_free = v_full + kDqVSlots;            // [kK]
+  uint64_t* s_full = k_free + kDqKSlots;            // [2]
+  uint64_t* dp_full = s_full + 2;                   // [2]
+  uint64_t* dp_free = dp_full + 2;
+  uint64_t* ds_full = dp_free + 1;                  // [2]
+  uint64_t* drain_bar = ds_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* skip_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -154,13 +158,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < kDqKSlots; ++s) mbar_init(&k_full[s], 1);
+    for (int s = 0; s < kDqKSlots; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_free[s], 1);
+    }
+    for (int s = 0; s < kDqVSlots; ++s) mbar_init(&v_full[s], 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&v_full[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&dp_full[s], 1);
       mbar_init(&ds_full[s], 8);
-      mbar_init(&dq_done[s], 1);
     }
     mbar_init(dp_free, 8);
     mbar_init(drain_bar, 1);
@@ -201,8 +207,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       DqKvIter kvi(p, it);
       for (int i = 0; i < T; ++i, kvi.next(p)) {
         const int kv0 = kvi.kv0(p);
-        // K_i takes the slot of K_{i-3}: free once dQ(i-3) completed
-        if (i >= kDqKSlots && !wait_bounded(&dq_done[(i - 3) & 1], ((i - 3) >> 1) & 1, ctl, kQSiteLoadK)) break;
+        // K_i takes the slot of K_{i-kK}: free once dQ(i-kK) completed
+        if (i >= kDqKSlots &&
+            !wait_bounded(&k_free[i % kDqKSlots], ((i / kDqKSlots) - 1) & 1, ctl, kQSiteLoadK)) break;
         {
           uint64_t* full = &k_full[i % kDqKSlots];
           uint8_t* dst = k_s + (i % kDqKSlots) * kTile;
@@ -211,11 +218,13 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           for (int x = 0; x < kBoxes; ++x) tma_load_4d(dst + x * kBoxBytes, &tm_k, full, x * 64, kv0, it.g, it.b, pol_kv);
           ++nk;
         }
-        // V_i takes the slot of V_{i-2}: free once dP(i-2) completed
-        if (i >= kDqVSlots && !wait_bounded(&dp_full[(i - 2) & 1], ((i - 2) >> 1) & 1, ctl, kQSiteLoadV)) break;
+        // V_i takes the slot of V_{i-kV}: free once dP(i-kV) completed (dp_full of that tile;
+        // it cannot run two phases ahead: dP(i) needs V_i)
+        if (i >= kDqVSlots && !wait_bounded(&dp_full[(i - kDqVSlots) & 1], ((i - kDqVSlots) >> 1) & 1, ctl,
+                                            kQSiteLoadV)) break;
         {
-          uint64_t* full = &v_full[i & 1];
-          uint8_t* dst = v_s + (i & 1) * kTile;
+          uint64_t* full = &v_full[i % kDqVSlots];
+          uint8_t* dst = v_s + (i % kDqVSlots) * kTile;
           mbar_arrive_expect_tx(full, kTile);
 #pragma unroll
           for (int x = 0; x < kBoxes; ++x) tma_load_4d(dst + x * kBoxBytes, &tm_v, full, x * 64, kv0, it.g, it.b, pol_kv);
@@ -226,7 +235,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       dq_wait_drain(q_full, 0, ctl);
       for (int n = (nk > kDqKSlots ? nk - kDqKSlots : 0); n < nk; ++n)
         dq_wait_drain(&k_full[n % kDqKSlots], (n / kDqKSlots) & 1, ctl);
-      for (int n = (nv > kDqVSlots ? nv - kDqVSlots : 0); n < nv; ++n) dq_wait_drain(&v_full[n & 1], (n >> 1) & 1, ctl);
+      for (int n = (nv > kDqVSlots ? nv - kDqVSlots : 0); n < nv; ++n)
+        dq_wait_drain(&v_full[n % kDqVSlots], (n / kDqVSlots) & 1, ctl);
     }
     __syncwarp();
   } else if (warp == kDqMmaWarp) {
@@ -244,9 +254,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
       };
       auto wait_k = [&](int i) { return wait_bounded(&k_full[i % kDqKSlots], (i / kDqKSlots) & 1, ctl, kQSiteMmaK); };
-      auto wait_v = [&](int i) { return wait_bounded(&v_full[i & 1], (i >> 1) & 1, ctl, kQSiteMmaV); };
+      auto wait_v = [&](int i) {
+        return wait_bounded(&v_full[i % kDqVSlots], (i / kDqVSlots) & 1, ctl, kQSiteMmaV);
+      };
       auto kaddr = [&](int i) { return k_a0 + (i % kDqKSlots) * kTile; };
-      auto vaddr = [&](int i) { return v_a0 + (i & 1) * kTile; };
+      auto vaddr = [&](int i) { return v_a0 + (i % kDqVSlots) * kTile; };
 
       bool ok = wait_bounded(q_full, 0, ctl, kQSiteMmaQ);
       if (ok && T > 0) {
@@ -283,7 +295,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         for (int kk = 0; kk < 8; ++kk)  // keys [16 kk, 16 kk + 16): written by warpgroup kk / 4
           umma_ts(tDQ, ds_t + 64u * (kk >> 2) + 8u * (kk & 3), make_sdesc(ka + kk * 2048, kBoxBytes, 1024), idesc_o,
                   (i > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&dq_done[i & 1]);
+        umma_commit(&k_free[i % kDqKSlots]);
       }
       // drain: all MMAs issued by this thread are complete before TMEM is freed
       umma_commit(drain_bar);
@@ -360,7 +372,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     }
     // epilogue: dQ * scale -> bf16, d columns of this warpgroup's half
     if (ok && T > 0 &&
-        __all_sync(0xffffffffu, wait_bounded(&dq_done[(T - 1) & 1], ((T - 1) >> 1) & 1, ctl, kQSiteDone))) {
+        __all_sync(0xffffffffu,
+                   wait_bounded(&k_free[(T - 1) % kDqKSlots], ((T - 1) / kDqKSlots) & 1, ctl, kQSiteDone))) {
       tc_fence_after();
       __nv_bfloat16* dst = p.dq + it.b * p.dq_sb + it.h * p.dq_sh + static_cast<long long>(q_row) * p.dq_sl;
 #pragma unroll
