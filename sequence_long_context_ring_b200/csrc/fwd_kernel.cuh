@@ -9,7 +9,8 @@
 // One CTA owns two 128-row query tiles (A, B) that stream the same KV tiles:
 //   * GQA (G even): two query heads of one KV group at the same rows;
 //   * otherwise:    two consecutive 128-row tiles of one head inside one chunk.
-// The KV tiles are visited in ring order: the diagonal chunk r first, then r-1, ..., 0.
+// The KV chunks are visited in ascending order (0, 1, ..., the diagonal chunk r last), the same
+// for every rank, so concurrent CTAs share K/V tiles in L2.
 // Within a work item the running (max, sum, O) state is carried across tiles, so the merge
 // of a finished chunk's partial into the accumulator happens at every chunk boundary as the
 // same rescale-and-add that joins two tiles: (O, LSE) (+) (O', LSE') with weights e^(LSE-m).
@@ -137,29 +138,38 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p) {
   return it;
 }
 
-// The KV tiles of an item in ring visit order, walked without divisions (this runs once per
-// tile on the softmax critical path): chunk j, tile tt inside it, tiles left in the chunk.
-//   fused, causal:     chunk r (its first n_diag tiles), then r-1, ..., 0 (all tiles)
-//   fused, non-causal: chunks r, r-1, ... (mod N), all tiles
+// The KV tiles of an item in visit order, walked without divisions (this runs once per tile
+// on the softmax critical path): chunk j, tile tt inside it, tiles left in the chunk.
+//   fused, causal:     chunks 0, 1, ..., r-1 (all tiles), then the diagonal chunk r (its first
+//                      n_diag tiles)
+//   fused, non-causal: chunks 0, 1, ..., N-1
 //   one ring step:     chunk step_chunk, the item's n_tiles tiles
+// Every rank visits the chunks in the same ascending order (a ring schedule in which the
+// chunk that arrives at step s is chunk s; the merged result does not depend on the order),
+// so CTAs that start together stream the same K/V tiles at the same time and share them
+// through L2.
 struct KvIter {
-  int j, tt, left;
+  int j, tt, left, last, last_len;
   __device__ __forceinline__ KvIter(const FwdParams& p, const Item& it) {
     tt = 0;
     if (p.step_rank >= 0) {
       j = p.step_chunk;
       left = it.n_tiles;
+      last = -1;
+      last_len = 0;
     } else {
-      j = it.r;
-      left = p.causal ? it.n_diag : p.tiles_per_chunk;
+      j = 0;
+      last = p.causal ? it.r : -1;
+      last_len = it.n_diag;
+      left = (last == 0) ? last_len : p.tiles_per_chunk;
     }
   }
   __device__ __forceinline__ void next(const FwdParams& p) {
     ++tt;
     if (--left == 0) {
       tt = 0;
-      left = p.tiles_per_chunk;
-      j = (j == 0 ? p.n_chunks : j) - 1;
+      ++j;
+      left = (j == last) ? last_len : p.tiles_per_chunk;
     }
   }
   __device__ __forceinline__ int kv0(const FwdParams& p) const { return j * p.chunk_len + tt * kBN; }
