@@ -215,6 +215,21 @@ def run_reference(args, w):
 
 
 # ------------------------------------------------------------------------------------------
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The largest of every rank's device time (the job is as slow as its slowest replica)."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Throughput of the whole job: every replica's FLOPs over the slowest replica's time."""
+    return world * flops_per_step * steps / (max_ms / 1e3) / 1e12
+
+
 def _time_ms(fn, stream, warmup=3, reps=10):
     """Median device time of fn() (CUDA events on `stream`, synchronised on both sides)."""
     import torch
@@ -396,11 +411,8 @@ def run_ours(args, w):
     st, word = plan.device_status(stream)
     if st != 0:
         raise RuntimeError(f"device status {st} (word {word:#x}) in the timed region")
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
-    value = world * flops * args.steps / (max_ms / 1e3) / 1e12
+    max_ms = max_over_ranks(total_ms, world, dev)
+    value = whole_job_tflops(flops, args.steps, world, max_ms)
 
     # ---- end-to-end through the public API with host buffers ----
     qh, kh, vh = (torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -422,10 +434,7 @@ def run_ours(args, w):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * flops * args.e2e_steps / (float(te.item()) / 1e3) / 1e12
+    e2e_value = whole_job_tflops(flops, args.e2e_steps, world, max_over_ranks(e2e_ms, world, dev))
     h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
 
