@@ -19,6 +19,7 @@ Modules:
   attention  full causal softmax attention with LSE (the plain definition), row-sampled form
   ring       per-(rank, step) chunk partials, the LSE merge, ring / Ulysses / 2D flows
   layout     Ulysses sequence<->head re-layout by index formula
+  split      zig-zag / striped / contiguous rank-to-sequence maps, ring and Ulysses under them
   backward   gradient of softmax attention from its definition
 
 Every pin of this oracle is listed in tests/test_oracle_*.py; there is no function here
@@ -28,10 +29,14 @@ from .attention import attention_full, attention_rows, forward_flops
 from .ring import chunk_partial, lse_merge, ring_attention, ulysses_attention, attention_2d
 from .layout import seq2head, head2seq
 from .backward import attention_backward, backward_rows_dq, backward_rows_dkdv
+from .split import (rank_positions, rank_order, shards_of_rank, step_pairs, ring_step_split,
+                    ring_attention_split, seq2head_split, head2seq_split, ulysses_attention_split)
 
 __all__ = [
     "attention_full", "attention_rows", "forward_flops",
     "chunk_partial", "lse_merge", "ring_attention", "ulysses_attention", "attention_2d",
     "seq2head", "head2seq",
     "attention_backward", "backward_rows_dq", "backward_rows_dkdv",
+    "rank_positions", "rank_order", "shards_of_rank", "step_pairs", "ring_step_split",
+    "ring_attention_split", "seq2head_split", "head2seq_split", "ulysses_attention_split",
 ]
