@@ -66,9 +66,20 @@ typedef enum { CP_BF16 = 0, CP_FP32 = 1 } cp_dtype_t;
  *   ring over n_cp context chunks per head group, inverse re-layout ([2D]). */
 typedef enum { CP_MODE_RING = 0, CP_MODE_ULYSSES = 1, CP_MODE_2D = 2 } cp_mode_t;
 
-/* Chunk-to-rank map.  CONTIGUOUS: rank r owns positions [r*c, (r+1)*c).  ZIGZAG ([CP] §5)
- * is reserved: cp_attn_plan returns CP_ERR_UNSUPPORTED for it. */
-typedef enum { CP_SPLIT_CONTIGUOUS = 0, CP_SPLIT_ZIGZAG = 1 } cp_split_t;
+/* Chunk-to-rank map ([CP] §5, "因果モデルの負荷分散": a contiguous split gives later ranks more
+ * causal work).  CONTIGUOUS: rank r owns positions [r*c, (r+1)*c).  The two-shard splits cut
+ * the sequence into 2N shards of w = c/2 positions and give each rank two, its local rows
+ * being its first shard followed by its second:
+ *   ZIGZAG   rank r holds shards r and 2N-1-r (the page's example: 8 shards, N = 4 ->
+ *            [x0,x7],[x1,x6],[x2,x5],[x3,x4]); every rank has the same causal work;
+ *   STRIPED  rank r holds shards r and r+N (the page's "striped ordering", read as two
+ *            shards per rank placed in stripes).
+ * Two-shard splits need L % (2 n_cp) == 0 and apply to RING and ULYSSES plans (TWO_D:
+ * CP_ERR_UNSUPPORTED).  In RING mode they define the virtual ranks of cp_ring_step;
+ * cp_attn_fwd/bwd on the head-major tensors compute the same global result for every split.
+ * In ULYSSES mode the sequence-major tensors are rank-major: rank s's local rows at
+ * [s*c, (s+1)*c).  LSE is in position order [B, Hq, L] in every case. */
+typedef enum { CP_SPLIT_CONTIGUOUS = 0, CP_SPLIT_ZIGZAG = 1, CP_SPLIT_STRIPED = 2 } cp_split_t;
 
 typedef struct {
   void* data;         /* device pointer                                    */
@@ -96,7 +107,8 @@ typedef struct {
 typedef struct cp_plan cp_plan_t;
 
 /* Validate `cfg` and build a plan (host only; touches no GPU).
- * Rules: B,Hq,Hkv,L,d,n_cp >= 1; Hq % Hkv == 0; d in {64, 128}; RING: n_hp == 1,
+ * Rules: B,Hq,Hkv,L,d,n_cp >= 1; Hq % Hkv == 0; d in {64, 128}; a two-shard split needs
+ * L % (2 n_cp) == 0 and is not supported for TWO_D; RING: n_hp == 1,
  * L % n_cp == 0.  ULYSSES: n_hp == 1, L % n_cp == 0, Hq % n_cp == 0 and Hkv % n_cp == 0 (the
  * head-parallel degree cannot exceed the KV-group count: [UL] "Ring AttentionとUlyssesの設計上の
  * 違い", [USP] §2).  TWO_D: L % (n_hp*n_cp) == 0, Hq % n_hp == 0, Hkv % n_hp == 0.
@@ -105,9 +117,9 @@ cp_status_t cp_attn_plan(const cp_attn_config_t* cfg, cp_plan_t** out);
 void cp_attn_plan_destroy(cp_plan_t* plan);
 
 /* Device workspace (bytes) that cp_attn_fwd (backward=0) or cp_attn_bwd (backward=1) need.
- * RING forward: 0.  ULYSSES/TWO_D forward: head-major copies of q, k, v, o.  Backward: an
- * fp32 dQ accumulator [B,Hq,L,d] and D = rowsum(dO*O) [B,Hq,L] (+ head-major copies of
- * q, k, v, dO, dq, dk, dv for ULYSSES/TWO_D).  Sizes include 256 B alignment padding. */
+ * RING forward: 0.  ULYSSES/TWO_D forward: head-major copies of q, k, v, o.  Backward:
+ * D = rowsum(dO*O) [B,Hq,L] fp32 (+ head-major copies of q, dO, k, v, dk, dv for
+ * ULYSSES/TWO_D, and of dq under a two-shard split).  Sizes include 256 B alignment padding. */
 cp_status_t cp_attn_workspace_size(const cp_plan_t* plan, int backward, size_t* bytes);
 
 /* Forward.  Each query of each virtual rank accumulates causal softmax attention over every
@@ -157,11 +169,24 @@ cp_status_t cp_layout_seq2head(int n_ranks, const cp_tensor_t* in, cp_tensor_t* 
 /* Exact inverse ([UL] step 4): in [B, H, L, d] -> out [B, L, H, d]. */
 cp_status_t cp_layout_head2seq(int n_ranks, const cp_tensor_t* in, cp_tensor_t* out, void* stream);
 
+/* The same all-to-all under a chunk-to-rank map ([CP] §5): in [B, L, H, d] is rank-major
+ * (rank s's local rows at [s*c, (s+1)*c), in its shards' order), out [B, H, L, d] is in
+ * position order:  out[b, h, pos_s(t), :] = in[b, s*c + t, h, :], pos_s(t) the global
+ * position of rank s's local row t.  CONTIGUOUS equals cp_layout_seq2head.  Two-shard splits
+ * need L % (2 n_ranks) == 0.  Bit-exact copy. */
+cp_status_t cp_layout_seq2head_split(int n_ranks, cp_split_t split, const cp_tensor_t* in, cp_tensor_t* out,
+                                     void* stream);
+/* Exact inverse of cp_layout_seq2head_split: in [B, H, L, d] -> out [B, L, H, d]. */
+cp_status_t cp_layout_head2seq_split(int n_ranks, cp_split_t split, const cp_tensor_t* in, cp_tensor_t* out,
+                                     void* stream);
+
 /* One ring step of rank `rank` at step `step` (RING plans): the partial attention of query
  * chunk r against KV chunk j = (rank - step) mod n_cp ([CP] ring step 2).
  * q, k, v: the full tensors as for cp_attn_fwd.  o_part [B,Hq,c,d] fp32 receives the
  * normalised partial P V / l, lse_part [B,Hq,c] fp32 its LSE.  A chunk wholly above the
- * causal diagonal yields O = 0, LSE = -inf (the merge identity). */
+ * causal diagonal yields O = 0, LSE = -inf (the merge identity).  Under a two-shard split
+ * rank r's c rows are its two shards (local order) and the KV rows are rank j's two shards;
+ * a query shard that sees neither KV shard gets the identity. */
 cp_status_t cp_ring_step(const cp_plan_t* plan, int rank, int step, const cp_tensor_t* q,
                          const cp_tensor_t* k, const cp_tensor_t* v, cp_tensor_t* o_part,
                          cp_tensor_t* lse_part, void* stream);
@@ -182,7 +207,9 @@ const char* cp_status_string(cp_status_t status);
 
 /* ---- host-only plan queries (no GPU needed) ---------------------------------------------- */
 /* Ring map: at `step`, rank `rank` holds KV chunk *chunk = (rank - step) mod N, which is
- * *kind = 0 (skipped: wholly above the diagonal), 1 (fully visible) or 2 (diagonal, masked). */
+ * *kind = 0 (skipped: wholly above the diagonal), 1 (fully visible) or 2 (diagonal, masked).
+ * Under a two-shard split *chunk is the KV rank and *kind is 2 at the diagonal step and 1
+ * otherwise (some shard pair is visible at every step). */
 cp_status_t cp_plan_step_chunk(const cp_plan_t* plan, int rank, int step, int* chunk, int* kind);
 /* Algorithmic FLOPs of one forward (4*B*Hq*d*visible pairs) or backward (2.5x forward). */
 cp_status_t cp_plan_flops(const cp_plan_t* plan, int backward, double* flops);

@@ -20,7 +20,7 @@ CP_OK, CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED, CP_ERR_ALIGNMENT = 0, -1, -2, -3
 CP_ERR_WORKSPACE, CP_ERR_CUDA, CP_ERR_TIMEOUT = -4, -5, -6
 CP_BF16, CP_FP32 = 0, 1
 MODES = {"ring": 0, "ulysses": 1, "2d": 2}
-SPLITS = {"contiguous": 0, "zigzag": 1}
+SPLITS = {"contiguous": 0, "zigzag": 1, "striped": 2}
 
 
 class CpError(RuntimeError):
@@ -45,7 +45,7 @@ EXPORTS = [
     "cp_attn_plan", "cp_attn_plan_destroy", "cp_attn_workspace_size", "cp_attn_fwd", "cp_attn_bwd",
     "cp_layout_seq2head", "cp_layout_head2seq", "cp_ring_step", "cp_lse_merge", "cp_device_status",
     "cp_status_string", "cp_plan_step_chunk", "cp_plan_flops", "cp_plan_num_work_items", "cp_version",
-    "cp_attn_fwd_noalloc",
+    "cp_attn_fwd_noalloc", "cp_layout_seq2head_split", "cp_layout_head2seq_split",
 ]
 
 
@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
             "cp_plan_num_work_items": ([P, ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
             "cp_version": ([], ctypes.c_char_p),
             "cp_attn_fwd_noalloc": ([P, T, T, T, T, T, P], ctypes.c_int),
+            "cp_layout_seq2head_split": ([ctypes.c_int, ctypes.c_int, T, T, P], ctypes.c_int),
+            "cp_layout_head2seq_split": ([ctypes.c_int, ctypes.c_int, T, T, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -226,21 +228,31 @@ def lse_merge(o_acc, lse_acc, o_part, lse_part, stream=None) -> None:
     _check(lib().cp_lse_merge(*[ctypes.byref(t) for t in td], _stream(stream)), "cp_lse_merge")
 
 
-def seq2head(n_ranks: int, x, out=None, stream=None):
-    """[B, L, H, d] -> [B, H, L, d] (Ulysses all-to-all, bit-exact)."""
+def seq2head(n_ranks: int, x, out=None, stream=None, split: str = "contiguous"):
+    """[B, L, H, d] (rank-major under a two-shard split) -> [B, H, L, d] in position order
+    (Ulysses all-to-all, bit-exact)."""
     if out is None:
         B, L, H, d = x.shape
         out = torch.empty((B, H, L, d), dtype=x.dtype, device=x.device)
     a, b = tensor_desc(x), tensor_desc(out)
-    _check(lib().cp_layout_seq2head(n_ranks, ctypes.byref(a), ctypes.byref(b), _stream(stream)), "cp_layout_seq2head")
+    if split == "contiguous":
+        _check(lib().cp_layout_seq2head(n_ranks, ctypes.byref(a), ctypes.byref(b), _stream(stream)), "cp_layout_seq2head")
+    else:
+        _check(lib().cp_layout_seq2head_split(n_ranks, SPLITS[split], ctypes.byref(a), ctypes.byref(b), _stream(stream)),
+               "cp_layout_seq2head_split")
     return out
 
 
-def head2seq(n_ranks: int, x, out=None, stream=None):
-    """[B, H, L, d] -> [B, L, H, d] (inverse all-to-all, bit-exact)."""
+def head2seq(n_ranks: int, x, out=None, stream=None, split: str = "contiguous"):
+    """[B, H, L, d] in position order -> [B, L, H, d] (rank-major under a two-shard split),
+    the inverse all-to-all, bit-exact."""
     if out is None:
         B, H, L, d = x.shape
         out = torch.empty((B, L, H, d), dtype=x.dtype, device=x.device)
     a, b = tensor_desc(x), tensor_desc(out)
-    _check(lib().cp_layout_head2seq(n_ranks, ctypes.byref(a), ctypes.byref(b), _stream(stream)), "cp_layout_head2seq")
+    if split == "contiguous":
+        _check(lib().cp_layout_head2seq(n_ranks, ctypes.byref(a), ctypes.byref(b), _stream(stream)), "cp_layout_head2seq")
+    else:
+        _check(lib().cp_layout_head2seq_split(n_ranks, SPLITS[split], ctypes.byref(a), ctypes.byref(b), _stream(stream)),
+               "cp_layout_head2seq_split")
     return out

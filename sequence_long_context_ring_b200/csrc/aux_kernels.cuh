@@ -22,7 +22,32 @@ struct PermuteParams {
   int X, Y;              // in is [B, X, Y, row]; out is [B, Y, X, row]
   long long in_sb, in_sx, in_sy;     // strides in 16-byte vectors
   long long out_sb, out_sy, out_sx;
+  // Two-shard splits: the sequence axis of the rank-major side is in rank order (rank s's
+  // rows at [s*c, (s+1)*c): its first shard, then its second), the other side in position
+  // order.  remap 1: the output's x is a position, the input's x its rank-major row;
+  // remap 2: the output's y is a rank-major row, the input's y its position.  0: none.
+  int remap, split, n_ranks, shard;  // split 1 zig-zag (shards r, 2N-1-r), 2 striped (r, r+N)
 };
+
+// Rank-major row of global position pos under a two-shard split (split 1 zig-zag, 2
+// striped; n ranks, shard length w = c / 2).
+__device__ __forceinline__ int split_rank_row(int pos, int split, int n, int w) {
+  const int sh = pos / w, off = pos - sh * w;
+  const int hi = sh >= n;  // the rank's second shard
+  const int r = hi ? (split == 1 ? 2 * n - 1 - sh : sh - n) : sh;
+  return r * 2 * w + hi * w + off;
+}
+__device__ __forceinline__ int rank_row_of_pos(const PermuteParams& p, int pos) {
+  return split_rank_row(pos, p.split, p.n_ranks, p.shard);
+}
+// Global position of rank-major row u.
+__device__ __forceinline__ int pos_of_rank_row(const PermuteParams& p, int u) {
+  const int w = p.shard, n = p.n_ranks;
+  const int r = u / (2 * w), t = u - r * 2 * w;
+  const int hi = t >= w;
+  const int sh = hi ? (p.split == 1 ? 2 * n - 1 - r : r + n) : r;
+  return sh * w + (t - hi * w);
+}
 
 constexpr int kPermThreads = 256;
 constexpr int kVecPerThread = 4;
@@ -43,7 +68,9 @@ __global__ void __launch_bounds__(kPermThreads) permute_rows_kernel(const Permut
       t /= p.X;
       const int y = static_cast<int>(t % p.Y);
       const long long b = t / p.Y;
-      v[u] = __ldg(p.in + b * p.in_sb + x * p.in_sx + y * p.in_sy + vec);
+      const int xi = p.remap == 1 ? rank_row_of_pos(p, x) : x;
+      const int yi = p.remap == 2 ? pos_of_rank_row(p, y) : y;
+      v[u] = __ldg(p.in + b * p.in_sb + xi * p.in_sx + yi * p.in_sy + vec);
       dst[u] = b * p.out_sb + y * p.out_sy + x * p.out_sx + vec;
     }
   }
@@ -113,6 +140,9 @@ struct DotParams {
   int B, H, L, d;
   long long o_sb, o_sh, o_sl, g_sb, g_sh, g_sl;  // element strides of o and dout ([b,h,l] axes)
   long long D_sb, D_sh, D_sl;
+  // D is in position order; under a two-shard split (split 1 zig-zag, 2 striped) the rows of
+  // o and dout are rank-major: position l is read from row split_rank_row(l).  0: same order.
+  int split, n_ranks, shard;
 };
 
 __global__ void __launch_bounds__(256) rowdot_kernel(const DotParams p) {
@@ -128,8 +158,9 @@ __global__ void __launch_bounds__(256) rowdot_kernel(const DotParams p) {
     l = static_cast<int>(row % p.L);
     h = static_cast<int>((row / p.L) % p.H);
     b = static_cast<int>(row / (static_cast<long long>(p.L) * p.H));
-    const uint4 a = reinterpret_cast<const uint4*>(p.o + b * p.o_sb + h * p.o_sh + l * p.o_sl)[vec];
-    const uint4 g = reinterpret_cast<const uint4*>(p.dout + b * p.g_sb + h * p.g_sh + l * p.g_sl)[vec];
+    const long long lr = p.split ? split_rank_row(l, p.split, p.n_ranks, p.shard) : l;
+    const uint4 a = reinterpret_cast<const uint4*>(p.o + b * p.o_sb + h * p.o_sh + lr * p.o_sl)[vec];
+    const uint4 g = reinterpret_cast<const uint4*>(p.dout + b * p.g_sb + h * p.g_sh + lr * p.g_sl)[vec];
     const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
     const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
 #pragma unroll

@@ -169,6 +169,7 @@ void fill_geometry(const cp_plan_t* plan, int n_chunks, FwdParams& p) {
   p.scale_log2 = static_cast<float>(static_cast<double>(plan->scale) * 1.4426950408889634);
   p.step_rank = -1;
   p.step_chunk = 0;
+  p.step_chunk2 = -1;
   p.out_row_base = 0;
   p.wait_limit_ns = c.wait_limit_ns ? c.wait_limit_ns : kDefaultWaitLimitNs;
   p.debug_fault = c.debug_fault;
@@ -201,7 +202,8 @@ cp_status_t run_fwd_kernel(const cp_plan_t* plan, FwdParams& p, const View& q, c
 // ---- permute ------------------------------------------------------------------------------
 // out[b, y, x, :] = in[b, x, y, :] for in [B, X, Y, d] (element strides given per axis).
 cp_status_t launch_permute(const void* in, void* out, int64_t B, int64_t X, int64_t Y, int64_t d, int eb,
-                           const int64_t in_str[3], const int64_t out_str_yx[3], cudaStream_t s) {
+                           const int64_t in_str[3], const int64_t out_str_yx[3], cudaStream_t s, int remap = 0,
+                           cp_split_t split = CP_SPLIT_CONTIGUOUS, int n_ranks = 1) {
   const int64_t row_bytes = d * eb;
   if (row_bytes % 16 != 0) return CP_ERR_ALIGNMENT;
   PermuteParams p;
@@ -218,6 +220,15 @@ cp_status_t launch_permute(const void* in, void* out, int64_t B, int64_t X, int6
   p.out_sb = out_str_yx[0] / per;
   p.out_sy = out_str_yx[1] / per;
   p.out_sx = out_str_yx[2] / per;
+  p.remap = (split == CP_SPLIT_CONTIGUOUS) ? 0 : remap;
+  p.split = split == CP_SPLIT_ZIGZAG ? 1 : 2;
+  p.n_ranks = n_ranks;
+  p.shard = 1;
+  if (p.remap) {
+    const int64_t L = remap == 1 ? X : Y;
+    if (n_ranks < 1 || L % (2 * n_ranks) != 0) return CP_ERR_INVALID_ARG;
+    p.shard = static_cast<int>(L / (2 * n_ranks));
+  }
   if (p.n_vec == 0) return CP_OK;
   const int64_t per_block = kPermThreads * kVecPerThread;
   const int64_t grid = (p.n_vec + per_block - 1) / per_block;
@@ -225,19 +236,22 @@ cp_status_t launch_permute(const void* in, void* out, int64_t B, int64_t X, int6
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
-// seq-major [B, L, H, d] tensor -> contiguous head-major buffer [B, H, L, d]
-cp_status_t seq_to_head_buf(const cp_tensor_t* in, void* buf, cudaStream_t s) {
+// seq-major [B, L, H, d] tensor (rank-major rows under a two-shard split) -> contiguous
+// head-major buffer [B, H, L, d] in position order
+cp_status_t seq_to_head_buf(const cp_tensor_t* in, void* buf, cudaStream_t s, cp_split_t split = CP_SPLIT_CONTIGUOUS,
+                            int n_ranks = 1) {
   const int64_t B = in->shape[0], L = in->shape[1], H = in->shape[2], d = in->shape[3];
   const int64_t in_str[3] = {in->stride[0], in->stride[1], in->stride[2]};
   const int64_t out_str[3] = {H * L * d, L * d, d};  // (b, y=h, x=l)
-  return launch_permute(in->data, buf, B, L, H, d, elem_bytes(in->dtype), in_str, out_str, s);
+  return launch_permute(in->data, buf, B, L, H, d, elem_bytes(in->dtype), in_str, out_str, s, 1, split, n_ranks);
 }
-// contiguous head-major buffer [B, H, L, d] -> seq-major tensor [B, L, H, d]
-cp_status_t head_buf_to_seq(const void* buf, cp_tensor_t* out, cudaStream_t s) {
+// contiguous head-major buffer [B, H, L, d] in position order -> seq-major tensor [B, L, H, d]
+cp_status_t head_buf_to_seq(const void* buf, cp_tensor_t* out, cudaStream_t s, cp_split_t split = CP_SPLIT_CONTIGUOUS,
+                            int n_ranks = 1) {
   const int64_t B = out->shape[0], L = out->shape[1], H = out->shape[2], d = out->shape[3];
   const int64_t in_str[3] = {H * L * d, L * d, d};                      // (b, x=h, y=l)
   const int64_t out_str[3] = {out->stride[0], out->stride[1], out->stride[2]};  // (b, y=l, x=h)
-  return launch_permute(buf, out->data, B, H, L, d, elem_bytes(out->dtype), in_str, out_str, s);
+  return launch_permute(buf, out->data, B, H, L, d, elem_bytes(out->dtype), in_str, out_str, s, 2, split, n_ranks);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -266,9 +280,12 @@ cp_status_t launch_bwd_dq_d(const DqParams& p, const CUtensorMap& mq, const CUte
 
 // D = rowsum(dO * O) for [b, h, l] rows given by per-axis element strides.
 cp_status_t launch_rowdot(const void* o, const int64_t os[3], const void* g, const int64_t gs[3], float* D, int B,
-                          int H, int L, int d, cudaStream_t s) {
+                          int H, int L, int d, cudaStream_t s, cp_split_t split = CP_SPLIT_CONTIGUOUS,
+                          int n_ranks = 1) {
+  const int sp = split == CP_SPLIT_ZIGZAG ? 1 : (split == CP_SPLIT_STRIPED ? 2 : 0);
   DotParams p{static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(g), D, B, H, L, d,
-              os[0], os[1], os[2], gs[0], gs[1], gs[2], (int64_t)H * L, (int64_t)L, 1};
+              os[0], os[1], os[2], gs[0], gs[1], gs[2], (int64_t)H * L, (int64_t)L, 1,
+              sp, n_ranks, sp ? L / (2 * n_ranks) : 1};
   const int64_t threads = (int64_t)B * H * L * (d / 8);
   if (threads == 0) return CP_OK;
   rowdot_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(p);
@@ -320,10 +337,12 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
   const int64_t os[3] = {o->stride[0], seq ? o->stride[2] : o->stride[1], seq ? o->stride[1] : o->stride[2]};
   const int64_t gs[3] = {dout->stride[0], seq ? dout->stride[2] : dout->stride[1],
                          seq ? dout->stride[1] : dout->stride[2]};
-  CP_TRY(launch_rowdot(o->data, os, dout->data, gs, Dvec, c.B, c.Hq, c.L, c.d, s));
+  CP_TRY(launch_rowdot(o->data, os, dout->data, gs, Dvec, c.B, c.Hq, c.L, c.d, s, seq ? c.split : CP_SPLIT_CONTIGUOUS,
+                       c.n_cp));
 
   View vq, vk, vv, vdo;
-  void *dkh = nullptr, *dvh = nullptr;
+  void *dkh = nullptr, *dvh = nullptr, *dqh = nullptr;
+  const bool remap = seq && c.split != CP_SPLIT_CONTIGUOUS;
   if (!seq) {
     vq = view_of(q);
     vk = view_of(k);
@@ -341,12 +360,14 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
     dkh = w;
     w += align256(nkv * 2);
     dvh = w;
+    w += align256(nkv * 2);
+    if (remap) dqh = w;  // under a two-shard split dQ goes head-major first, then rank-major
     // all-to-all seq -> head of the inputs and of the upstream gradient (the extra a2a of the
     // backward, "05. 長系列の分散学習（Context Parallelism）" §3)
-    CP_TRY(seq_to_head_buf(q, qh, s));
-    CP_TRY(seq_to_head_buf(k, kh, s));
-    CP_TRY(seq_to_head_buf(v, vh, s));
-    CP_TRY(seq_to_head_buf(dout, doh, s));
+    CP_TRY(seq_to_head_buf(q, qh, s, c.split, c.n_cp));
+    CP_TRY(seq_to_head_buf(k, kh, s, c.split, c.n_cp));
+    CP_TRY(seq_to_head_buf(v, vh, s, c.split, c.n_cp));
+    CP_TRY(seq_to_head_buf(dout, doh, s, c.split, c.n_cp));
     vq = contiguous_view(qh, c.B, c.Hq, c.L, c.d);
     vk = contiguous_view(kh, c.B, c.Hkv, c.L, c.d);
     vv = contiguous_view(vh, c.B, c.Hkv, c.L, c.d);
@@ -420,10 +441,17 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
   qp.lse_sh = p.lse_sh;
   qp.lse_sl = p.lse_sl;
   qp.Dvec = Dvec;
-  qp.dq = static_cast<__nv_bfloat16*>(dq->data);
-  qp.dq_sb = dq->stride[0];
-  qp.dq_sh = seq ? dq->stride[2] : dq->stride[1];
-  qp.dq_sl = seq ? dq->stride[1] : dq->stride[2];
+  if (remap) {
+    qp.dq = static_cast<__nv_bfloat16*>(dqh);
+    qp.dq_sb = (int64_t)c.Hq * c.L * c.d;
+    qp.dq_sh = (int64_t)c.L * c.d;
+    qp.dq_sl = c.d;
+  } else {
+    qp.dq = static_cast<__nv_bfloat16*>(dq->data);
+    qp.dq_sb = dq->stride[0];
+    qp.dq_sh = seq ? dq->stride[2] : dq->stride[1];
+    qp.dq_sl = seq ? dq->stride[1] : dq->stride[2];
+  }
   qp.status = sw;
   qp.wait_limit_ns = p.wait_limit_ns;
   const int64_t qgrid = (int64_t)qp.n_chunks * qp.tiles_per_chunk * c.B * c.Hq;
@@ -433,9 +461,10 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
     CP_TRY(launch_bwd_dq_d<64>(qp, mq, mk, mv, mdo, qgrid, s));
   }
   if (!seq) return CP_OK;
-  // all-to-all head -> seq of dK and dV
-  CP_TRY(head_buf_to_seq(dkh, dk, s));
-  return head_buf_to_seq(dvh, dv, s);
+  // all-to-all head -> seq of dK and dV (and of dQ under a two-shard split)
+  if (remap) CP_TRY(head_buf_to_seq(dqh, dq, s, c.split, c.n_cp));
+  CP_TRY(head_buf_to_seq(dkh, dk, s, c.split, c.n_cp));
+  return head_buf_to_seq(dvh, dv, s, c.split, c.n_cp);
 }
 
 }  // namespace
@@ -465,8 +494,12 @@ cp_status_t cp_attn_plan(const cp_attn_config_t* cfg, cp_plan_t** out) {
   if (c.Hq % c.Hkv != 0) return CP_ERR_INVALID_ARG;
   if (c.causal != 0 && c.causal != 1) return CP_ERR_INVALID_ARG;
   if (!(c.softmax_scale >= 0.f) || std::isinf(c.softmax_scale)) return CP_ERR_INVALID_ARG;
-  if (c.split == CP_SPLIT_ZIGZAG) return CP_ERR_UNSUPPORTED;
-  if (c.split != CP_SPLIT_CONTIGUOUS) return CP_ERR_INVALID_ARG;
+  if (c.split != CP_SPLIT_CONTIGUOUS && c.split != CP_SPLIT_ZIGZAG && c.split != CP_SPLIT_STRIPED)
+    return CP_ERR_INVALID_ARG;
+  if (c.split != CP_SPLIT_CONTIGUOUS) {
+    if (c.mode == CP_MODE_2D) return CP_ERR_UNSUPPORTED;
+    if (c.n_cp < 1 || c.L % (2 * c.n_cp) != 0) return CP_ERR_INVALID_ARG;  // two shards per rank
+  }
   switch (c.mode) {
     case CP_MODE_RING:
       if (c.n_hp != 1 || c.L % c.n_cp != 0) return CP_ERR_INVALID_ARG;
@@ -516,6 +549,7 @@ cp_status_t cp_attn_workspace_size(const cp_plan_t* plan, int backward, size_t* 
   } else {
     ws = align256(nrow * 4);                                             // D
     if (seq_major) ws += 2 * align256(nq * 2) + 4 * align256(nkv * 2);  // q, do ; k, v, dk, dv
+    if (seq_major && c.split != CP_SPLIT_CONTIGUOUS) ws += align256(nq * 2);  // dq
   }
   *bytes = ws;
   return CP_OK;
@@ -558,9 +592,9 @@ cp_status_t cp_attn_fwd(const cp_plan_t* plan, const cp_tensor_t* q, const cp_te
   w += align256(nkv * 2);
   void* oh = w;
   // step 2 of the Ulysses flow (head-group all-to-all for 2D): seq -> head
-  CP_TRY(seq_to_head_buf(q, qh, s));
-  CP_TRY(seq_to_head_buf(k, kh, s));
-  CP_TRY(seq_to_head_buf(v, vh, s));
+  CP_TRY(seq_to_head_buf(q, qh, s, c.split, c.n_cp));
+  CP_TRY(seq_to_head_buf(k, kh, s, c.split, c.n_cp));
+  CP_TRY(seq_to_head_buf(v, vh, s, c.split, c.n_cp));
   // step 3: attention per head group (Ulysses: one chunk = full sequence; 2D: ring over n_cp)
   fill_geometry(plan, c.mode == CP_MODE_ULYSSES ? 1 : c.n_cp, p);
   const int64_t grid = (int64_t)p.n_chunks * p.pos_per_chunk * p.n_inner;
@@ -569,7 +603,7 @@ cp_status_t cp_attn_fwd(const cp_plan_t* plan, const cp_tensor_t* q, const cp_te
   CP_TRY(run_fwd_kernel(plan, p, contiguous_view(qh, c.B, c.Hq, c.L, c.d), contiguous_view(kh, c.B, c.Hkv, c.L, c.d),
                         contiguous_view(vh, c.B, c.Hkv, c.L, c.d), out, grid, s));
   // step 4: head -> seq
-  return head_buf_to_seq(oh, o, s);
+  return head_buf_to_seq(oh, o, s, c.split, c.n_cp);
 }
 
 cp_status_t cp_ring_step(const cp_plan_t* plan, int rank, int step, const cp_tensor_t* q, const cp_tensor_t* k,
@@ -587,6 +621,46 @@ cp_status_t cp_ring_step(const cp_plan_t* plan, int rank, int step, const cp_ten
   CP_TRY(check3(lse_part, c.B, c.Hq, ch));
   const cudaStream_t s = as_stream(stream);
   const int j = ((rank - step) % N + N) % N;
+  if (c.split != CP_SPLIT_CONTIGUOUS) {
+    // Two shards per rank (each w = c/2 rows), chunks of a 2N-chunk split: the query rows are
+    // rank's shards (a0, a1) in that order, the KV rows rank j's shards (b0, b1).  One launch
+    // per query shard covers both KV shards, merged in the kernel; a query shard that sees
+    // neither gets the merge identity.
+    const int w = ch / 2;
+    auto shards = [&](int r, int& x0, int& x1) {
+      x0 = r;
+      x1 = c.split == CP_SPLIT_ZIGZAG ? 2 * N - 1 - r : r + N;
+    };
+    int a[2], b[2];
+    shards(rank, a[0], a[1]);
+    shards(j, b[0], b[1]);
+    for (int hq = 0; hq < 2; ++hq) {
+      int vis[2], nv = 0;
+      for (int t = 0; t < 2; ++t)
+        if (!c.causal || b[t] <= a[hq]) vis[nv++] = b[t];
+      if (nv == 0) {
+        const int64_t n = (int64_t)c.B * c.Hq * w * c.d;
+        fill_identity_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+            static_cast<float*>(o_part->data) + (int64_t)hq * w * o_part->stride[2],
+            static_cast<float*>(lse_part->data) + (int64_t)hq * w * lse_part->stride[2], c.B, c.Hq, w, c.d,
+            o_part->stride[0], o_part->stride[1], o_part->stride[2], lse_part->stride[0], lse_part->stride[1],
+            lse_part->stride[2]);
+        if (cudaGetLastError() != cudaSuccess) return CP_ERR_CUDA;
+        continue;
+      }
+      FwdParams p{};
+      fill_geometry(plan, 2 * N, p);
+      p.step_rank = a[hq];
+      p.step_chunk = vis[0];
+      p.step_chunk2 = nv > 1 ? vis[1] : -1;
+      p.out_row_base = (a[hq] - hq) * w;  // query shard a[hq] lands at rows [hq*w, (hq+1)*w)
+      const int64_t grid = (int64_t)p.pos_per_chunk * p.n_inner;
+      FwdOut out{o_part->data, o_part->stride[0], o_part->stride[1], o_part->stride[2], 1,
+                 static_cast<float*>(lse_part->data), lse_part->stride[0], lse_part->stride[1], lse_part->stride[2]};
+      CP_TRY(run_fwd_kernel(plan, p, view_of(q), view_of(k), view_of(v), out, grid, s));
+    }
+    return CP_OK;
+  }
   if (c.causal && j > rank) {
     const int64_t n = (int64_t)c.B * c.Hq * ch * c.d;
     fill_identity_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
@@ -652,6 +726,36 @@ cp_status_t cp_layout_head2seq(int n_ranks, const cp_tensor_t* in, cp_tensor_t* 
   return launch_permute(in->data, out->data, B, H, L, d, elem_bytes(in->dtype), in_str, out_str, as_stream(stream));
 }
 
+cp_status_t cp_layout_seq2head_split(int n_ranks, cp_split_t split, const cp_tensor_t* in, cp_tensor_t* out,
+                                     void* stream) {
+  if (!in || !out || n_ranks < 1) return CP_ERR_INVALID_ARG;
+  if (split != CP_SPLIT_CONTIGUOUS && split != CP_SPLIT_ZIGZAG && split != CP_SPLIT_STRIPED) return CP_ERR_INVALID_ARG;
+  const int64_t B = in->shape[0], L = in->shape[1], H = in->shape[2], d = in->shape[3];
+  if (in->dtype != out->dtype) return CP_ERR_INVALID_ARG;
+  CP_TRY(check4(in, in->dtype, B, L, H, d));
+  CP_TRY(check4(out, out->dtype, B, H, L, d));
+  if (H % n_ranks != 0 || L % (split == CP_SPLIT_CONTIGUOUS ? n_ranks : 2 * n_ranks) != 0) return CP_ERR_INVALID_ARG;
+  const int64_t in_str[3] = {in->stride[0], in->stride[1], in->stride[2]};
+  const int64_t out_str[3] = {out->stride[0], out->stride[1], out->stride[2]};  // (b, y=h, x=l)
+  return launch_permute(in->data, out->data, B, L, H, d, elem_bytes(in->dtype), in_str, out_str, as_stream(stream), 1,
+                        split, n_ranks);
+}
+
+cp_status_t cp_layout_head2seq_split(int n_ranks, cp_split_t split, const cp_tensor_t* in, cp_tensor_t* out,
+                                     void* stream) {
+  if (!in || !out || n_ranks < 1) return CP_ERR_INVALID_ARG;
+  if (split != CP_SPLIT_CONTIGUOUS && split != CP_SPLIT_ZIGZAG && split != CP_SPLIT_STRIPED) return CP_ERR_INVALID_ARG;
+  const int64_t B = in->shape[0], H = in->shape[1], L = in->shape[2], d = in->shape[3];
+  if (in->dtype != out->dtype) return CP_ERR_INVALID_ARG;
+  CP_TRY(check4(in, in->dtype, B, H, L, d));
+  CP_TRY(check4(out, out->dtype, B, L, H, d));
+  if (H % n_ranks != 0 || L % (split == CP_SPLIT_CONTIGUOUS ? n_ranks : 2 * n_ranks) != 0) return CP_ERR_INVALID_ARG;
+  const int64_t in_str[3] = {in->stride[0], in->stride[1], in->stride[2]};
+  const int64_t out_str[3] = {out->stride[0], out->stride[1], out->stride[2]};  // (b, y=l, x=h)
+  return launch_permute(in->data, out->data, B, H, L, d, elem_bytes(in->dtype), in_str, out_str, as_stream(stream), 2,
+                        split, n_ranks);
+}
+
 cp_status_t cp_device_status(const cp_plan_t* plan, void* stream, int* detail) {
   if (!plan) return CP_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return CP_ERR_CUDA;
@@ -680,6 +784,11 @@ cp_status_t cp_plan_step_chunk(const cp_plan_t* plan, int rank, int step, int* c
   if (rank < 0 || rank >= N || step < 0 || step >= N) return CP_ERR_INVALID_ARG;
   const int j = ((rank - step) % N + N) % N;
   *chunk = j;
+  if (c.split != CP_SPLIT_CONTIGUOUS) {
+    // two shards per rank: some shard of rank j is below some shard of `rank` at every step
+    *kind = !c.causal ? 1 : (j == rank ? 2 : 1);
+    return CP_OK;
+  }
   *kind = !c.causal ? 1 : (j > rank ? 0 : (j == rank ? 2 : 1));
   return CP_OK;
 }
@@ -768,9 +877,9 @@ extern "C" cp_status_t cp_attn_fwd_noalloc(const cp_plan_t* plan, const cp_tenso
   void* oh = w;
   // Every byte of the scratch that is read below is written first in this call, so nothing
   // from an earlier call needs clearing.
-  CP_TRY(seq_to_head_buf(q, qh, s));
-  CP_TRY(seq_to_head_buf(k, kh, s));
-  CP_TRY(seq_to_head_buf(v, vh, s));
+  CP_TRY(seq_to_head_buf(q, qh, s, c.split, c.n_cp));
+  CP_TRY(seq_to_head_buf(k, kh, s, c.split, c.n_cp));
+  CP_TRY(seq_to_head_buf(v, vh, s, c.split, c.n_cp));
   FwdParams p{};
   fill_geometry(plan, c.mode == CP_MODE_ULYSSES ? 1 : c.n_cp, p);
   p.o = oh;
@@ -795,5 +904,5 @@ extern "C" cp_status_t cp_attn_fwd_noalloc(const cp_plan_t* plan, const cp_tenso
       CP_TRY(launch_fwd_d<64>(p, mq, mk, mv, grid, s));
     }
   }
-  return head_buf_to_seq(oh, o, s);
+  return head_buf_to_seq(oh, o, s, c.split, c.n_cp);
 }

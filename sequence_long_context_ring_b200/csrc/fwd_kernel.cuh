@@ -73,8 +73,10 @@ struct FwdParams {
   int n_inner;               // work items per query position
   int causal;
   float scale_log2;          // softmax scale * log2(e)
-  int step_rank;             // -1: fused over all ranks and steps; else one (rank, chunk) step
-  int step_chunk;
+  int step_rank;             // -1: fused over all ranks and steps; else one step: query chunk
+  int step_chunk;            // step_rank against KV chunk step_chunk and, when step_chunk2 >= 0,
+  int step_chunk2;           // also chunk step_chunk2 (the two shards a rank holds under a
+                             // two-shard split), merged in the kernel
   int out_row_base;          // subtracted from the global row when writing o / lse
   void* o;                   // bf16 or fp32 output, [B, Hq, rows, d]
   long long o_sb, o_sh, o_sl;
@@ -89,6 +91,13 @@ struct FwdParams {
 struct Item {
   int b, g, headA, headB, rowA, rowB, r, q_end, n_tiles, n_diag;
 };
+
+// KV tiles of chunk b that the query tiles of item it (in chunk it.r) see in one step.
+__device__ __forceinline__ int step_tiles(const FwdParams& p, int r, int n_diag, int b) {
+  if (b < 0) return 0;
+  if (!p.causal) return p.tiles_per_chunk;
+  return b < r ? p.tiles_per_chunk : (b == r ? n_diag : 0);
+}
 
 __device__ __forceinline__ Item decode_item(const FwdParams& p) {
   Item it;
@@ -129,7 +138,7 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p) {
   }
   it.n_diag = (last - c0) / kBN + 1;
   if (p.step_rank >= 0) {
-    it.n_tiles = (p.causal && p.step_chunk == it.r) ? it.n_diag : p.tiles_per_chunk;
+    it.n_tiles = step_tiles(p, it.r, it.n_diag, p.step_chunk) + step_tiles(p, it.r, it.n_diag, p.step_chunk2);
   } else if (p.causal) {
     it.n_tiles = it.n_diag + it.r * p.tiles_per_chunk;
   } else {
@@ -143,18 +152,32 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p) {
 //   fused, causal:     chunks 0, 1, ..., r-1 (all tiles), then the diagonal chunk r (its first
 //                      n_diag tiles)
 //   fused, non-causal: chunks 0, 1, ..., N-1
-//   one ring step:     chunk step_chunk, the item's n_tiles tiles
+//   one ring step:     chunk step_chunk, then chunk step_chunk2 if set (each only as far as
+//                      the causal mask lets the item's query tiles see it)
 // Every rank visits the chunks in the same ascending order (a ring schedule in which the
 // chunk that arrives at step s is chunk s; the merged result does not depend on the order),
 // so CTAs that start together stream the same K/V tiles at the same time and share them
 // through L2.
 struct KvIter {
-  int j, tt, left, last, last_len;
+  int j, tt, left, last, last_len, second, second_len;
   __device__ __forceinline__ KvIter(const FwdParams& p, const Item& it) {
     tt = 0;
+    second = -1;
+    second_len = 0;
     if (p.step_rank >= 0) {
-      j = p.step_chunk;
-      left = it.n_tiles;
+      const int t1 = step_tiles(p, it.r, it.n_diag, p.step_chunk);
+      const int t2 = step_tiles(p, it.r, it.n_diag, p.step_chunk2);
+      if (t1 > 0) {
+        j = p.step_chunk;
+        left = t1;
+        if (t2 > 0) {
+          second = p.step_chunk2;
+          second_len = t2;
+        }
+      } else {
+        j = p.step_chunk2;
+        left = t2;
+      }
       last = -1;
       last_len = 0;
     } else {
@@ -168,8 +191,14 @@ struct KvIter {
     ++tt;
     if (--left == 0) {
       tt = 0;
-      ++j;
-      left = (j == last) ? last_len : p.tiles_per_chunk;
+      if (second >= 0) {
+        j = second;
+        left = second_len;
+        second = -1;
+      } else {
+        ++j;
+        left = (j == last) ? last_len : p.tiles_per_chunk;
+      }
     }
   }
   __device__ __forceinline__ int kv0(const FwdParams& p) const { return j * p.chunk_len + tt * kBN; }

@@ -51,7 +51,9 @@ def test_version_and_status_strings():
     (dict(mode="ulysses", n_cp=3, L=999), binding.CP_ERR_INVALID_ARG),   # H % N != 0
     (dict(mode="ulysses", Hq=32, Hkv=4, n_cp=8), binding.CP_ERR_INVALID_ARG),  # degree > KV groups
     (dict(mode="2d", n_hp=3, n_cp=2), binding.CP_ERR_INVALID_ARG),       # Hq % n_hp != 0
-    (dict(split="zigzag"), binding.CP_ERR_UNSUPPORTED),
+    (dict(mode="2d", n_hp=2, n_cp=2, split="zigzag"), binding.CP_ERR_UNSUPPORTED),  # 2D: contiguous only
+    (dict(split="zigzag", L=1028, n_cp=4), binding.CP_ERR_INVALID_ARG),   # two shards per rank: 2N | L
+    (dict(split="striped", mode="ulysses", L=1020, n_cp=4), binding.CP_ERR_INVALID_ARG),
     (dict(B=0), binding.CP_ERR_INVALID_ARG),
 ])
 def test_plan_validation_errors(kw, err):
@@ -77,6 +79,19 @@ def test_ring_map_and_skip_set():
         p.step_chunk(4, 0)
     nc = Plan(B=1, Hq=4, Hkv=4, L=1024, d=64, n_cp=4, causal=False)
     assert all(nc.step_chunk(r, s)[1] == 1 for r in range(4) for s in range(4))
+
+
+@pytest.mark.parametrize("split", ["zigzag", "striped"])
+def test_two_shard_splits_plan_and_ring_map(split):
+    # ring and Ulysses plans accept the two-shard splits; at every ring step some shard of the
+    # KV rank is visible to some shard of the query rank, the diagonal step holds masked blocks
+    Plan(B=1, Hq=8, Hkv=8, L=1024, d=128, n_cp=4, mode="ulysses", split=split)
+    p = Plan(B=1, Hq=8, Hkv=8, L=1024, d=128, n_cp=4, split=split)
+    for r in range(4):
+        for s in range(4):
+            j, kind = p.step_chunk(r, s)
+            assert j == (r - s) % 4
+            assert kind == (2 if j == r else 1)
 
 
 def test_flops_and_work_items():
