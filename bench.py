@@ -286,6 +286,9 @@ def measure_rows(dev, peaks, l_div: int = 1):
     nbytes = 2 * x.numel() * 2
     hbm_row("seq2head", f"c4 shape [1,{L},32,128] bf16", _time_ms(lambda: binding.seq2head(w.n_cp, x, y), stream), nbytes)
     hbm_row("head2seq", f"c4 shape [1,32,{L},128] bf16", _time_ms(lambda: binding.head2seq(w.n_cp, y, x), stream), nbytes)
+    # the same all-to-all with zig-zag rank-major rows (row remap between rank and position order)
+    hbm_row("seq2head_zigzag", f"c4 shape [1,{L},32,128] bf16, zig-zag split",
+            _time_ms(lambda: binding.seq2head(w.n_cp, x, y, split="zigzag"), stream), nbytes)
     del y
     # a6: Ulysses forward, c4 (seq->head, attention per head group, head->seq)
     k, v = rnd(w.B, L, w.Hkv, w.d), rnd(w.B, L, w.Hkv, w.d)
@@ -328,6 +331,10 @@ def measure_rows(dev, peaks, l_div: int = 1):
     tc_row("ring_step", f"c2 rank {r} step 1 (full chunk {r - 1} of {ch} keys)",
            _time_ms(lambda: plan.ring_step(r, 1, q, k, v, po, pl, stream), stream),
            4.0 * w.B * w.Hq * w.d * ch * ch)
+    zplan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp, split="zigzag")
+    tc_row("ring_step_zigzag", f"c2 zig-zag rank {r} step 1 (two query shards x two KV shards)",
+           _time_ms(lambda: zplan.ring_step(r, 1, q, k, v, po, pl, stream), stream),
+           4.0 * w.B * w.Hq * w.d * (2 * (ch // 2) * (ch // 2)))
     acc_o = torch.zeros_like(po)
     acc_l = torch.full_like(pl, -float("inf"))
     hbm_row("lse_merge", f"c2 chunk [1,32,{ch},128] fp32",
