@@ -248,13 +248,15 @@ def _time_ms(fn, stream, warmup=3, reps=10):
 def measure_rows(dev, peaks, l_div: int = 1):
     """Device time of every other step of the hot path at its workload's shape (random bf16
     device inputs; no host data): the Ulysses permutes and the Ulysses forward (c4 shape), the
-    2D forward and backward (c5 shape), the ring backward (c2 shape), and one step-wise ring
-    step plus its LSE merge (c2 shape).  Each entry carries its roofline: HBM-bound steps
-    against the measured copy bandwidth, contractions against the measured bf16 peak."""
+    2D forward and backward (c5 shape), the ring backward (c2 shape), one step-wise ring
+    step plus its LSE merge (c2 shape), and the point-to-point FIR convolution with a short
+    and a medium filter (c3's sequence and chunking, 4096 channels).  Each entry carries its
+    roofline: HBM-bound steps against the measured copy bandwidth, contractions against the
+    measured bf16 peak."""
     import torch
     from sequence_long_context_ring_b200 import binding
-    from sequence_long_context_ring_b200.binding import Plan
-    from sequence_long_context_ring_b200.configs import WORKLOADS
+    from sequence_long_context_ring_b200.binding import ConvPlan, Plan
+    from sequence_long_context_ring_b200.configs import CONV_WORKLOADS, WORKLOADS
 
     hbm = float(peaks["hbm_gbs"])
     tc = float(peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained")))
@@ -344,6 +346,23 @@ def measure_rows(dev, peaks, l_div: int = 1):
     st, word = plan.device_status(stream)
     if st != 0:
         raise RuntimeError(f"device status {st} ({word:#x}) in the row measurements")
+    del q, k, v, do, o, lse, wsb, dq, dk, dv, po, pl, acc_o, acc_l, plan, zplan
+    # point-to-point FIR convolution over all 16 virtual ranks (halos read in place): x read
+    # once, y written once (1.7 GB each at full size, well above L2)
+    for key in ("fir_short", "fir_medium"):
+        w = CONV_WORKLOADS[key]
+        L = w.L // l_div
+        x = rnd(w.B, w.D, L)
+        h = (rnd(w.D, w.lh).float() * w.h_scale).to(torch.bfloat16)
+        y = torch.empty_like(x)
+        cplan = ConvPlan(w.B, w.D, L, w.lh, w.n_cp)
+        hbm_row(key, f"[1,{w.D},{L}] bf16, l_h={w.lh}, N_cp={w.n_cp}",
+                _time_ms(lambda: cplan.fwd(x, h, y, stream), stream), cplan.cost()[0])
+        torch.cuda.synchronize()
+        st, word = cplan.device_status(stream)
+        if st != 0:
+            raise RuntimeError(f"device status {st} ({word:#x}) in the {key} row")
+        del x, h, y, cplan
     return rows
 
 

@@ -1,6 +1,6 @@
 """ctypes binding of libcpattn.so (argument marshalling only: every step runs in the CUDA kernels).
 
-Names follow the C ABI in include/cp_attn.h.  torch tensors are passed as strided views
+Names follow the C ABI in include/cp_attn.h and include/cp_conv.h.  torch tensors are passed as strided views
 (data pointer, shape, strides in elements); streams default to torch's current stream.
 There is no fallback: if the library is missing or a call fails, an exception is raised.
 """
@@ -41,11 +41,18 @@ class CpConfig(ctypes.Structure):
                 ("wait_limit_ns", ctypes.c_uint64), ("debug_fault", ctypes.c_int)]
 
 
+class ConvConfig(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("D", ctypes.c_int), ("L", ctypes.c_int), ("lh", ctypes.c_int),
+                ("n_cp", ctypes.c_int), ("wait_limit_ns", ctypes.c_uint64)]
+
+
 EXPORTS = [
     "cp_attn_plan", "cp_attn_plan_destroy", "cp_attn_workspace_size", "cp_attn_fwd", "cp_attn_bwd",
     "cp_layout_seq2head", "cp_layout_head2seq", "cp_ring_step", "cp_lse_merge", "cp_device_status",
     "cp_status_string", "cp_plan_step_chunk", "cp_plan_flops", "cp_plan_num_work_items", "cp_version",
     "cp_attn_fwd_noalloc", "cp_layout_seq2head_split", "cp_layout_head2seq_split",
+    "cp_conv_plan", "cp_conv_plan_destroy", "cp_conv_fir_fwd", "cp_conv_fir_shard", "cp_conv_device_status",
+    "cp_conv_cost",
 ]
 
 
@@ -77,6 +84,12 @@ def lib() -> ctypes.CDLL:
             "cp_attn_fwd_noalloc": ([P, T, T, T, T, T, P], ctypes.c_int),
             "cp_layout_seq2head_split": ([ctypes.c_int, ctypes.c_int, T, T, P], ctypes.c_int),
             "cp_layout_head2seq_split": ([ctypes.c_int, ctypes.c_int, T, T, P], ctypes.c_int),
+            "cp_conv_plan": ([ctypes.POINTER(ConvConfig), ctypes.POINTER(ctypes.c_void_p)], ctypes.c_int),
+            "cp_conv_plan_destroy": ([P], None),
+            "cp_conv_fir_fwd": ([P, T, T, T, P], ctypes.c_int),
+            "cp_conv_fir_shard": ([P, ctypes.c_int, T, T, T, T, P], ctypes.c_int),
+            "cp_conv_device_status": ([P, P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
+            "cp_conv_cost": ([P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -92,15 +105,15 @@ def _check(status: int, what: str) -> None:
 
 
 def tensor_desc(t: torch.Tensor) -> CpTensor:
-    """Strided-view descriptor of a device tensor (bf16 or fp32, 3-D or 4-D)."""
+    """Strided-view descriptor of a device tensor (bf16 or fp32, 2-D to 4-D)."""
     if t.dtype == torch.bfloat16:
         dt = CP_BF16
     elif t.dtype == torch.float32:
         dt = CP_FP32
     else:
         raise TypeError(f"unsupported dtype {t.dtype}")
-    if t.dim() not in (3, 4):
-        raise ValueError("expected a 3-D or 4-D tensor")
+    if t.dim() not in (2, 3, 4):
+        raise ValueError("expected a 2-D, 3-D or 4-D tensor")
     d = CpTensor()
     d.data = t.data_ptr()
     d.dtype = dt
@@ -256,3 +269,47 @@ def head2seq(n_ranks: int, x, out=None, stream=None, split: str = "contiguous"):
         _check(lib().cp_layout_head2seq_split(n_ranks, SPLITS[split], ctypes.byref(a), ctypes.byref(b), _stream(stream)),
                "cp_layout_head2seq_split")
     return out
+
+
+class ConvPlan:
+    """A cp_conv plan: the causal depthwise FIR convolution of a sequence sharded over n_cp
+    contiguous virtual ranks (include/cp_conv.h)."""
+
+    def __init__(self, B: int, D: int, L: int, lh: int, n_cp: int = 1, wait_limit_ns: int = 0):
+        self.cfg = ConvConfig(B, D, L, lh, n_cp, int(wait_limit_ns))
+        h = ctypes.c_void_p()
+        _check(lib().cp_conv_plan(ctypes.byref(self.cfg), ctypes.byref(h)), "cp_conv_plan")
+        self._h = h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.cp_conv_plan_destroy(h)
+            self._h = None
+
+    def cost(self):
+        """(HBM bytes, multiply-adds) of one whole-sequence convolution."""
+        b, f = ctypes.c_double(), ctypes.c_double()
+        _check(lib().cp_conv_cost(self._h, ctypes.byref(b), ctypes.byref(f)), "cp_conv_cost")
+        return b.value, f.value
+
+    def fwd(self, x, h, y=None, stream=None):
+        """y = x * h over the whole sequence [B, D, L] (every virtual rank, halos in place)."""
+        y = torch.empty_like(x) if y is None else y
+        td = [tensor_desc(t) for t in (x, h, y)]
+        _check(lib().cp_conv_fir_fwd(self._h, *[ctypes.byref(t) for t in td], _stream(stream)), "cp_conv_fir_fwd")
+        return y
+
+    def shard(self, rank: int, x, halo, h, y=None, stream=None):
+        """One rank's shard [B, D, L/n_cp] with the halo [B, D, lh-1] from rank-1 (None at rank 0)."""
+        y = torch.empty_like(x) if y is None else y
+        dx, dh, dy = tensor_desc(x), tensor_desc(h), tensor_desc(y)
+        dg = ctypes.byref(tensor_desc(halo)) if halo is not None else None
+        _check(lib().cp_conv_fir_shard(self._h, int(rank), ctypes.byref(dx), dg, ctypes.byref(dh),
+                                       ctypes.byref(dy), _stream(stream)), "cp_conv_fir_shard")
+        return y
+
+    def device_status(self, stream=None):
+        detail = ctypes.c_int()
+        st = lib().cp_conv_device_status(self._h, _stream(stream), ctypes.byref(detail))
+        return st, detail.value

@@ -8,9 +8,9 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libcpattn.so")
-SOURCES = [os.path.join(PKG, "csrc", "cp_attn.cu")]
+SOURCES = [os.path.join(PKG, "csrc", "cp_attn.cu"), os.path.join(PKG, "csrc", "cp_conv.cu")]
 DEPS = SOURCES + [os.path.join(PKG, "csrc", f) for f in os.listdir(os.path.join(PKG, "csrc"))] + [
-    os.path.join(ROOT, "include", "cp_attn.h")]
+    os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -6,6 +6,12 @@
   c3  long-context Llama-3-8B-shaped GQA ring attention: L=212992 (208K), N_cp=16 (13312)
   c4  Ulysses, 7B-MHA: H=32, d=128, L=131072, degree 8; sequence-major per-rank input
   c5  2D head x context grid 4 x 4, 7B-MHA: H=32, d=128, L=65536, forward + backward
+
+Point-to-point FIR convolution ("05. 長系列の分散学習（Context Parallelism）" §3), on c3's
+sequence and chunking at the Llama-3-8B width (D = 4096 channels):
+  fir_short   l_h = 7 taps    (a short explicit filter: halo of 6 samples per rank)
+  fir_medium  l_h = 128 taps  (a medium filter: halo of 127 samples per rank)
+Inputs: x ~ N(0, 1), h ~ N(0, 1/l_h), both rounded to bf16.
 """
 from __future__ import annotations
 
@@ -49,4 +55,31 @@ WORKLOADS = {
     "c3": Workload("c3_llama3_8b_gqa_L212992_N16", 3, 1, 32, 8, 212992, 128, 16, 1, "ring"),
     "c4": Workload("c4_ulysses_7b_mha_L131072_N8", 4, 1, 32, 32, 131072, 128, 8, 1, "ulysses"),
     "c5": Workload("c5_2d_4x4_7b_mha_L65536_fwd_bwd", 5, 1, 32, 32, 65536, 128, 4, 4, "2d", backward=True),
+}
+
+
+@dataclass(frozen=True)
+class ConvWorkload:
+    name: str
+    cfg_id: int
+    B: int
+    D: int
+    L: int
+    lh: int
+    n_cp: int
+
+    def x_shape(self):
+        return (self.B, self.D, self.L)
+
+    def h_shape(self):
+        return (self.D, self.lh)
+
+    @property
+    def h_scale(self) -> float:
+        return self.lh ** -0.5
+
+
+CONV_WORKLOADS = {
+    "fir_short": ConvWorkload("fir_short_D4096_L212992_N16_lh7", 6, 1, 4096, 212992, 7, 16),
+    "fir_medium": ConvWorkload("fir_medium_D4096_L212992_N16_lh128", 7, 1, 4096, 212992, 128, 16),
 }

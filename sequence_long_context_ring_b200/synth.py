@@ -1,11 +1,11 @@
 """Seeded synthetic inputs shared by the CUDA path's tests/bench and the CPU oracle.
 
-This module holds no attention arithmetic: it only draws i.i.d. normal values from a
+This module holds no attention or convolution arithmetic: it only draws i.i.d. normal values from a
 fixed seed and rounds them to bfloat16.  Both sides of every parity check read the same
 host arrays produced here.
 
 Generator: numpy ``Generator(PCG64)`` seeded with ``default_rng([cfg_id, tensor_id])``;
-tensor ids are Q=0, K=1, V=2, dO=3.  Values are float32 ``standard_normal`` (drawn in
+tensor ids are Q=0, K=1, V=2, dO=3, and for the convolution x=4, h=5.  Values are float32 ``standard_normal`` (drawn in
 blocks of at most 64 Mi elements to bound host memory), multiplied by ``scale`` in
 float32, then rounded to bf16 by round-to-nearest-even on the bit pattern.
 """
@@ -13,7 +13,7 @@ from __future__ import annotations
 
 import numpy as np
 
-TENSOR_ID = {"q": 0, "k": 1, "v": 2, "do": 3}
+TENSOR_ID = {"q": 0, "k": 1, "v": 2, "do": 3, "x": 4, "h": 5}
 _BLOCK = 1 << 26  # elements per float32 draw (256 MiB)
 
 
