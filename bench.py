@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements of the other hot-path steps")
     ap.add_argument("--rows-only", action="store_true", help="measure only the other hot-path steps (one JSON line)")
     ap.add_argument("--rows-l-div", type=int, default=1, help="divide each row's sequence length (small ncu cases)")
+    ap.add_argument("--row", action="append", default=[], help="with --rows-only: measure only this row (repeatable)")
     return ap.parse_args()
 
 
@@ -245,14 +246,14 @@ def _time_ms(fn, stream, warmup=3, reps=10):
     return statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(reps))
 
 
-def measure_rows(dev, peaks, l_div: int = 1):
+def measure_rows(dev, peaks, l_div: int = 1, only=None):
     """Device time of every other step of the hot path at its workload's shape (random bf16
     device inputs; no host data): the Ulysses permutes and the Ulysses forward (c4 shape), the
     2D forward and backward (c5 shape), the ring backward (c2 shape), one step-wise ring
     step plus its LSE merge (c2 shape), and the point-to-point FIR convolution with a short
     and a medium filter (c3's sequence and chunking, 4096 channels).  Each entry carries its
     roofline: HBM-bound steps against the measured copy bandwidth, contractions against the
-    measured bf16 peak."""
+    measured bf16 peak.  `only`: a set of row names to measure (None: all)."""
     import torch
     from sequence_long_context_ring_b200 import binding
     from sequence_long_context_ring_b200.binding import ConvPlan, Plan
@@ -280,89 +281,99 @@ def measure_rows(dev, peaks, l_div: int = 1):
                       "roofline": {"bound": "tensor", "achieved": tf, "peak": tc, "unit": "TFLOP/s", "frac": tf / tc,
                                    "flops": flops}}
 
-    # a4 / a5: Ulysses re-layout at the c4 shape (one 1 GiB tensor each way)
-    w = WORKLOADS["c4"]
-    L = w.L // l_div
-    x = rnd(w.B, L, w.Hq, w.d)
-    y = torch.empty((w.B, w.Hq, L, w.d), dtype=torch.bfloat16, device=dev)
-    nbytes = 2 * x.numel() * 2
-    hbm_row("seq2head", f"c4 shape [1,{L},32,128] bf16", _time_ms(lambda: binding.seq2head(w.n_cp, x, y), stream), nbytes)
-    hbm_row("head2seq", f"c4 shape [1,32,{L},128] bf16", _time_ms(lambda: binding.head2seq(w.n_cp, y, x), stream), nbytes)
-    # the same all-to-all with zig-zag rank-major rows (row remap between rank and position order)
-    hbm_row("seq2head_zigzag", f"c4 shape [1,{L},32,128] bf16, zig-zag split",
-            _time_ms(lambda: binding.seq2head(w.n_cp, x, y, split="zigzag"), stream), nbytes)
-    del y
-    # a6: Ulysses forward, c4 (seq->head, attention per head group, head->seq)
-    k, v = rnd(w.B, L, w.Hkv, w.d), rnd(w.B, L, w.Hkv, w.d)
-    plan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp, mode="ulysses")
-    o = torch.empty_like(x)
-    lse = torch.empty((w.B, w.Hq, L), dtype=torch.float32, device=dev)
-    ws = plan.workspace(False, dev)
-    tc_row("ulysses_fwd", f"c4 L={L} degree 8", _time_ms(lambda: plan.fwd(x, k, v, o, lse, ws, stream), stream, reps=5),
-           plan.flops(False))
-    del x, k, v, o, lse, ws, plan
-    # 2D forward and backward, c5
-    w = WORKLOADS["c5"]
-    L = w.L // l_div
-    q, k, v, do = rnd(w.B, L, w.Hq, w.d), rnd(w.B, L, w.Hkv, w.d), rnd(w.B, L, w.Hkv, w.d), rnd(w.B, L, w.Hq, w.d)
-    plan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp, n_hp=w.n_hp, mode="2d")
-    o = torch.empty_like(q)
-    lse = torch.empty((w.B, w.Hq, L), dtype=torch.float32, device=dev)
-    ws = plan.workspace(False, dev)
-    tc_row("2d_fwd", f"c5 L={L} grid 4x4", _time_ms(lambda: plan.fwd(q, k, v, o, lse, ws, stream), stream, reps=5),
-           plan.flops(False))
-    wsb = plan.workspace(True, dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    tc_row("2d_bwd", f"c5 L={L} grid 4x4 (D preprocess, a2a of q/k/v/dO, kernel, dQ cast, a2a back)",
-           _time_ms(lambda: plan.bwd(q, k, v, o, lse, do, dq, dk, dv, wsb, stream), stream, reps=5), plan.flops(True))
-    del q, k, v, do, o, lse, ws, wsb, dq, dk, dv, plan
-    # ring backward and the step-wise path at the c2 shape
-    w = WORKLOADS["c2"]
-    L = w.L // l_div
-    q, k, v, do = rnd(w.B, w.Hq, L, w.d), rnd(w.B, w.Hkv, L, w.d), rnd(w.B, w.Hkv, L, w.d), rnd(w.B, w.Hq, L, w.d)
-    plan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp)
-    o, lse = plan.fwd(q, k, v)
-    wsb = plan.workspace(True, dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    tc_row("ring_bwd", f"c2 L={L} N=8 (D preprocess, kernel, dQ cast)",
-           _time_ms(lambda: plan.bwd(q, k, v, o, lse, do, dq, dk, dv, wsb, stream), stream, reps=5), plan.flops(True))
-    ch = L // w.n_cp
-    po = torch.empty((w.B, w.Hq, ch, w.d), dtype=torch.float32, device=dev)
-    pl = torch.empty((w.B, w.Hq, ch), dtype=torch.float32, device=dev)
-    r = w.n_cp - 1
-    tc_row("ring_step", f"c2 rank {r} step 1 (full chunk {r - 1} of {ch} keys)",
-           _time_ms(lambda: plan.ring_step(r, 1, q, k, v, po, pl, stream), stream),
-           4.0 * w.B * w.Hq * w.d * ch * ch)
-    zplan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp, split="zigzag")
-    tc_row("ring_step_zigzag", f"c2 zig-zag rank {r} step 1 (two query shards x two KV shards)",
-           _time_ms(lambda: zplan.ring_step(r, 1, q, k, v, po, pl, stream), stream),
-           4.0 * w.B * w.Hq * w.d * (2 * (ch // 2) * (ch // 2)))
-    acc_o = torch.zeros_like(po)
-    acc_l = torch.full_like(pl, -float("inf"))
-    hbm_row("lse_merge", f"c2 chunk [1,32,{ch},128] fp32",
-            _time_ms(lambda: binding.lse_merge(acc_o, acc_l, po, pl, stream), stream),
-            (3 * po.numel() + 3 * pl.numel()) * 4)
-    torch.cuda.synchronize()
-    st, word = plan.device_status(stream)
-    if st != 0:
-        raise RuntimeError(f"device status {st} ({word:#x}) in the row measurements")
-    del q, k, v, do, o, lse, wsb, dq, dk, dv, po, pl, acc_o, acc_l, plan, zplan
-    # point-to-point FIR convolution over all 16 virtual ranks (halos read in place): x read
-    # once, y written once (1.7 GB each at full size, well above L2)
-    for key in ("fir_short", "fir_medium"):
-        w = CONV_WORKLOADS[key]
+    groups = {"ulysses": ("seq2head", "head2seq", "seq2head_zigzag", "ulysses_fwd"), "2d": ("2d_fwd", "2d_bwd"),
+              "ring": ("ring_bwd", "ring_step", "ring_step_zigzag", "lse_merge"), "fir": ("fir_short", "fir_medium")}
+    want = lambda grp: only is None or any(n in only for n in groups[grp])
+
+    if want("ulysses"):
+        # a4 / a5: Ulysses re-layout at the c4 shape (one 1 GiB tensor each way)
+        w = WORKLOADS["c4"]
         L = w.L // l_div
-        x = rnd(w.B, w.D, L)
-        h = (rnd(w.D, w.lh).float() * w.h_scale).to(torch.bfloat16)
-        y = torch.empty_like(x)
-        cplan = ConvPlan(w.B, w.D, L, w.lh, w.n_cp)
-        hbm_row(key, f"[1,{w.D},{L}] bf16, l_h={w.lh}, N_cp={w.n_cp}",
-                _time_ms(lambda: cplan.fwd(x, h, y, stream), stream), cplan.cost()[0])
+        x = rnd(w.B, L, w.Hq, w.d)
+        y = torch.empty((w.B, w.Hq, L, w.d), dtype=torch.bfloat16, device=dev)
+        nbytes = 2 * x.numel() * 2
+        hbm_row("seq2head", f"c4 shape [1,{L},32,128] bf16", _time_ms(lambda: binding.seq2head(w.n_cp, x, y), stream), nbytes)
+        hbm_row("head2seq", f"c4 shape [1,32,{L},128] bf16", _time_ms(lambda: binding.head2seq(w.n_cp, y, x), stream), nbytes)
+        # the same all-to-all with zig-zag rank-major rows (row remap between rank and position order)
+        hbm_row("seq2head_zigzag", f"c4 shape [1,{L},32,128] bf16, zig-zag split",
+                _time_ms(lambda: binding.seq2head(w.n_cp, x, y, split="zigzag"), stream), nbytes)
+        del y
+        # a6: Ulysses forward, c4 (seq->head, attention per head group, head->seq)
+        k, v = rnd(w.B, L, w.Hkv, w.d), rnd(w.B, L, w.Hkv, w.d)
+        plan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp, mode="ulysses")
+        o = torch.empty_like(x)
+        lse = torch.empty((w.B, w.Hq, L), dtype=torch.float32, device=dev)
+        ws = plan.workspace(False, dev)
+        tc_row("ulysses_fwd", f"c4 L={L} degree 8", _time_ms(lambda: plan.fwd(x, k, v, o, lse, ws, stream), stream, reps=5),
+               plan.flops(False))
+        del x, k, v, o, lse, ws, plan
+
+    if want("2d"):
+        # 2D forward and backward, c5
+        w = WORKLOADS["c5"]
+        L = w.L // l_div
+        q, k, v, do = rnd(w.B, L, w.Hq, w.d), rnd(w.B, L, w.Hkv, w.d), rnd(w.B, L, w.Hkv, w.d), rnd(w.B, L, w.Hq, w.d)
+        plan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp, n_hp=w.n_hp, mode="2d")
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, L), dtype=torch.float32, device=dev)
+        ws = plan.workspace(False, dev)
+        tc_row("2d_fwd", f"c5 L={L} grid 4x4", _time_ms(lambda: plan.fwd(q, k, v, o, lse, ws, stream), stream, reps=5),
+               plan.flops(False))
+        wsb = plan.workspace(True, dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        tc_row("2d_bwd", f"c5 L={L} grid 4x4 (D preprocess, a2a of q/k/v/dO, kernel, dQ cast, a2a back)",
+               _time_ms(lambda: plan.bwd(q, k, v, o, lse, do, dq, dk, dv, wsb, stream), stream, reps=5), plan.flops(True))
+        del q, k, v, do, o, lse, ws, wsb, dq, dk, dv, plan
+
+    if want("ring"):
+        # ring backward and the step-wise path at the c2 shape
+        w = WORKLOADS["c2"]
+        L = w.L // l_div
+        q, k, v, do = rnd(w.B, w.Hq, L, w.d), rnd(w.B, w.Hkv, L, w.d), rnd(w.B, w.Hkv, L, w.d), rnd(w.B, w.Hq, L, w.d)
+        plan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp)
+        o, lse = plan.fwd(q, k, v)
+        wsb = plan.workspace(True, dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        tc_row("ring_bwd", f"c2 L={L} N=8 (D preprocess, kernel, dQ cast)",
+               _time_ms(lambda: plan.bwd(q, k, v, o, lse, do, dq, dk, dv, wsb, stream), stream, reps=5), plan.flops(True))
+        ch = L // w.n_cp
+        po = torch.empty((w.B, w.Hq, ch, w.d), dtype=torch.float32, device=dev)
+        pl = torch.empty((w.B, w.Hq, ch), dtype=torch.float32, device=dev)
+        r = w.n_cp - 1
+        tc_row("ring_step", f"c2 rank {r} step 1 (full chunk {r - 1} of {ch} keys)",
+               _time_ms(lambda: plan.ring_step(r, 1, q, k, v, po, pl, stream), stream),
+               4.0 * w.B * w.Hq * w.d * ch * ch)
+        zplan = Plan(w.B, w.Hq, w.Hkv, L, w.d, n_cp=w.n_cp, split="zigzag")
+        tc_row("ring_step_zigzag", f"c2 zig-zag rank {r} step 1 (two query shards x two KV shards)",
+               _time_ms(lambda: zplan.ring_step(r, 1, q, k, v, po, pl, stream), stream),
+               4.0 * w.B * w.Hq * w.d * (2 * (ch // 2) * (ch // 2)))
+        acc_o = torch.zeros_like(po)
+        acc_l = torch.full_like(pl, -float("inf"))
+        hbm_row("lse_merge", f"c2 chunk [1,32,{ch},128] fp32",
+                _time_ms(lambda: binding.lse_merge(acc_o, acc_l, po, pl, stream), stream),
+                (3 * po.numel() + 3 * pl.numel()) * 4)
         torch.cuda.synchronize()
-        st, word = cplan.device_status(stream)
+        st, word = plan.device_status(stream)
         if st != 0:
-            raise RuntimeError(f"device status {st} ({word:#x}) in the {key} row")
-        del x, h, y, cplan
+            raise RuntimeError(f"device status {st} ({word:#x}) in the row measurements")
+
+    if want("fir"):
+        # point-to-point FIR convolution over all 16 virtual ranks (halos read in place): x read
+        # once, y written once (1.7 GB each at full size, well above L2)
+        for key in [k for k in ("fir_short", "fir_medium") if only is None or k in only]:
+            w = CONV_WORKLOADS[key]
+            L = w.L // l_div
+            x = rnd(w.B, w.D, L)
+            h = (rnd(w.D, w.lh).float() * w.h_scale).to(torch.bfloat16)
+            y = torch.empty_like(x)
+            cplan = ConvPlan(w.B, w.D, L, w.lh, w.n_cp)
+            hbm_row(key, f"[1,{w.D},{L}] bf16, l_h={w.lh}, N_cp={w.n_cp}",
+                    _time_ms(lambda: cplan.fwd(x, h, y, stream), stream), cplan.cost()[0])
+            torch.cuda.synchronize()
+            st, word = cplan.device_status(stream)
+            if st != 0:
+                raise RuntimeError(f"device status {st} ({word:#x}) in the {key} row")
+            del x, h, y, cplan
     return rows
 
 
@@ -371,7 +382,7 @@ def run_rows_only(args):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     peaks, src = load_peaks()
-    rows = measure_rows(dev, peaks, args.rows_l_div)
+    rows = measure_rows(dev, peaks, args.rows_l_div, set(args.row) if args.row else None)
     print(json.dumps({"rows": rows, "peaks": src, "rows_l_div": args.rows_l_div}), flush=True)
     return 0
 

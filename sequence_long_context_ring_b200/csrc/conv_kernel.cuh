@@ -12,18 +12,24 @@
 //   T0[i, j] = h[i - j]        (0 <= i - j < l_h)
 //   T1[i, j] = h[i - j + 128]  (i - j + 128 < l_h)
 //
-// i.e. two dense 128 x 128 x 128 contractions per block tile, with the two banded Toeplitz
-// matrices of the channel's filter as the B operand (built in shared memory once per channel)
-// and the input blocks as the A operand (K-major: a block is a contiguous 256-byte row).  The
-// previous-block operand is the same tensor read one block earlier; block -1 lies outside
-// the tensor map, so TMA fills it with zeros: the zero halo of rank 0, and the first stage of
-// the page's overlap variant.  Half of each Toeplitz pair is zero, which the tensor cores
-// absorb: the kernel stays bound by HBM (32 KB in + 32 KB out per 128 x 128 tile against
-// ~1000 tensor cycles), where the direct form at l_h = 128 would need 128 FMAs per output on
-// the CUDA cores, several times the HBM time.
+// i.e. two dense 128 x 128 x 128 contractions per block tile into one fp32 accumulator, with
+// the channel's banded Toeplitz pair as the B operand (built in shared memory once per
+// channel) and the input blocks as the A operand (K-major: a block is a contiguous 256-byte
+// row).  A stage holds the tile's 128 blocks preceded by 8 more (one 136-row TMA box per
+// 64-column half), so the previous-block operand X[m - 1] is the same buffer read one row
+// earlier: a descriptor starting 128 bytes before a 1024-byte swizzle atom.  The 128-byte
+// swizzle is a function of the absolute shared-memory address on both sides (TMA writes and
+// tcgen05 reads), so such a start needs no base offset (checked on the device against the
+// oracle: base offset 0 is exact, the other seven phases are not).  Blocks before the row's
+// start are outside the tensor map
+// and arrive as zeros: the zero halo of rank 0, and the first stage of the page's overlap
+// variant.  Half of each Toeplitz pair is zero, which the tensor cores absorb: the kernel
+// stays bound by HBM (32 KB in + 32 KB out per tile against at most ~1000 tensor cycles),
+// where the direct form at l_h = 128 would need 128 FMAs per output on the CUDA cores,
+// several times the HBM time.
 //
 // Roles (192 threads, one CTA per SM, persistent over a contiguous range of tiles):
-//   warp 0      TMA producer: current and previous blocks of a tile into a stage ring
+//   warp 0      TMA producer: the input rows of each block tile into a stage ring
 //   warp 1      TMEM owner and MMA issuer (two 128-column fp32 accumulators)
 //   warps 2-5   Toeplitz builder (at each channel change) and epilogue: TMEM -> bf16 ->
 //               128B-swizzled staging -> TMA store
@@ -76,8 +82,11 @@ __device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
 
 constexpr int kConvThreads = 192;
 constexpr int kConvMaxTaps = 129;                  // l_h - 1 <= 128: the halo fits one block
+constexpr int kConvLead = 8;                       // blocks loaded ahead of a tile's first
 constexpr uint32_t kConvBox = 128 * 64 * 2;        // 16 KB: 128 rows x 64 bf16, 128B swizzle
+constexpr uint32_t kConvInBox = (128 + kConvLead) * 128;   // 17 KB: a 136-row input half
 constexpr uint32_t kConvTmemCols = 256;
+constexpr int kRevLen = 392;                       // reversed filter copy: 49 x 8 entries
 enum : int { kCSiteLoad = 1, kCSiteMmaT = 2, kCSiteMmaX = 3, kCSiteMmaAcc = 4, kCSiteEpi = 5, kCSiteDrain = 7 };
 
 struct ConvParams {
@@ -85,25 +94,27 @@ struct ConvParams {
   int tiles_per_row;         // ceil(nblk / 128), nblk = 128-sample blocks of a row
   long long n_tiles;         // B * D * tiles_per_row
   int lh;                    // filter taps
+  int kk1;                   // first K step (16 samples) where T1 has taps: (129 - lh) / 16
   const __nv_bfloat16* h;    // filters [D, lh]
   long long h_sd;            // channel stride of h (elements)
   int* status;
   unsigned long long wait_limit_ns;
 };
 
-// Shared-memory plan for NPREV boxes of the previous-block operand (1: l_h <= 65, only its
-// columns 64..127 carry taps; 2: l_h <= 129).
-template <int NPREV>
+// Shared-memory plan.  Three input stages: measured at the full-size workloads, two leave
+// HBM idle between tiles and four lose bandwidth to the extra requests in flight.
 struct ConvSmem {
-  static constexpr int kStages = NPREV == 1 ? 3 : 2;
-  static constexpr uint32_t kStageBytes = (2 + NPREV) * kConvBox;
+  static constexpr int kStages = 3;
+  static constexpr uint32_t kStageBytes = 2 * kConvInBox;
+  static constexpr uint32_t kRevBytes = 8 * kRevLen * 2;
   static constexpr uint32_t kT0 = 0;
   static constexpr uint32_t kT1 = 2 * kConvBox;
-  static constexpr uint32_t kStage0 = kT1 + NPREV * kConvBox;
+  static constexpr uint32_t kStage0 = kT1 + 2 * kConvBox;
   static constexpr uint32_t kOut = kStage0 + kStages * kStageBytes;
-  static constexpr uint32_t kFilt = kOut + 2 * kConvBox;          // 256 bf16, zero-padded filter
+  static constexpr uint32_t kRev = kOut + 2 * kConvBox;          // 2 x 8 shifted reversed filters
+  static constexpr uint32_t kFilt = kRev + 2 * kRevBytes;        // 256 bf16, zero-padded filter
   static constexpr uint32_t kBars = kFilt + 512;
-  static constexpr uint32_t kBytes = kBars + 256;                  // after 1 KB alignment
+  static constexpr uint32_t kBytes = kBars + 256;                // after 1 KB alignment
 };
 
 // Shared-memory byte offset of element (r, col) of a 128-row tile held as two 128B-swizzled
@@ -123,22 +134,22 @@ __device__ __forceinline__ void conv_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
-template <int NPREV>
 __global__ void __launch_bounds__(kConvThreads, 1)
     fir_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
                   const ConvParams p) {
-  using S = ConvSmem<NPREV>;
+  using S = ConvSmem;
   constexpr int kStages = S::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint16_t* rev = reinterpret_cast<uint16_t*>(smem + S::kRev);
   uint16_t* filt = reinterpret_cast<uint16_t*>(smem + S::kFilt);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBars);
   // Barriers.  Tile i (local index) uses stage i % kStages and accumulator i & 1.
-  //  full[s]    TMA -> MMA: both operands of the stage landed (fill n = i / kStages, parity n & 1)
+  //  full[s]    TMA -> MMA: the stage's input rows landed (fill n = i / kStages, parity n & 1)
   //  empty[s]   MMA commit: the stage's MMAs completed, the producer may refill it
   //  tfull[a]   MMA commit: accumulator a holds tile i (parity (i >> 1) & 1)
   //  tempty[a]  epilogue -> MMA: accumulator a drained (one arrival per epilogue warp)
-  //  t_ready    builder -> MMA: the Toeplitz pair of the next channel is in shared memory
+  //  t_ready    builder -> MMA: the Toeplitz pair of the next row's channel is in shared memory
   //  drain      MMA commit at the end: all MMAs complete before TMEM is freed
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
@@ -201,15 +212,11 @@ __global__ void __launch_bounds__(kConvThreads, 1)
         const int row = static_cast<int>(t / p.tiles_per_row);
         const int m0 = static_cast<int>(t - static_cast<long long>(row) * p.tiles_per_row) * 128;
         const int b = row / p.D, ch = row - b * p.D;
-        uint8_t* cur = smem + S::kStage0 + s * S::kStageBytes;
-        uint8_t* prev = cur + 2 * kConvBox;
+        uint8_t* st = smem + S::kStage0 + s * S::kStageBytes;
+        // blocks m0 - 8 .. m0 + 127 (those before the row start arrive as zeros)
         mbar_arrive_expect_tx(&full[s], S::kStageBytes);
-        tma_load_4d(cur, &tm_x, &full[s], 0, m0, ch, b, pol);
-        tma_load_4d(cur + kConvBox, &tm_x, &full[s], 64, m0, ch, b, pol);
-        // block m0 - 1 of the row (zeros at m0 = 0); only the columns that carry taps
-#pragma unroll
-        for (int x = 0; x < NPREV; ++x)
-          tma_load_4d(prev + x * kConvBox, &tm_x, &full[s], (2 - NPREV + x) * 64, m0 - 1, ch, b, pol);
+        tma_load_4d(st, &tm_x, &full[s], 0, m0 - kConvLead, ch, b, pol);
+        tma_load_4d(st + kConvInBox, &tm_x, &full[s], 64, m0 - kConvLead, ch, b, pol);
         ++issued;
       }
       // drain: every load issued has landed before the CTA can exit
@@ -221,7 +228,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc_bf16(128, 128, false);
-      const int kk_prev = p.lh > 1 ? 8 - 4 * NPREV : 8;   // K steps of the previous block
+      const int kk_prev = p.lh > 1 ? p.kk1 : 8;       // K steps of the previous block with taps
       int rebuilds = 0, last_row = -1;
       bool ok = true;
       for (int i = 0; i < n_local && ok; ++i) {
@@ -237,17 +244,19 @@ __global__ void __launch_bounds__(kConvThreads, 1)
         if (i >= 2 && !wait_bounded(&tempty[a], ((i >> 1) - 1) & 1, ctl, kCSiteMmaAcc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem_base + a * 128;
-        const uint32_t cur = smem0 + S::kStage0 + s * S::kStageBytes;
-        const uint32_t prev = cur + 2 * kConvBox;
+        const uint32_t cur = smem0 + S::kStage0 + s * S::kStageBytes + kConvLead * 128;   // atom-aligned
+        const uint32_t prev = cur - 128;                                                   // one row earlier
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kConvBox + (kk & 3) * 32;
-          umma_ss(d, make_sdesc(cur + off, 16, 1024), make_sdesc(smem0 + S::kT0 + off, 16, 1024), idesc,
+          const uint32_t off = (kk >> 2) * kConvInBox + (kk & 3) * 32;
+          const uint32_t toff = (kk >> 2) * kConvBox + (kk & 3) * 32;
+          umma_ss(d, make_sdesc(cur + off, 16, 1024), make_sdesc(smem0 + S::kT0 + toff, 16, 1024), idesc,
                   kk > 0 ? 1u : 0u);
         }
         for (int kk = kk_prev; kk < 8; ++kk) {
-          const uint32_t off = ((kk >> 2) - (2 - NPREV)) * kConvBox + (kk & 3) * 32;
-          umma_ss(d, make_sdesc(prev + off, 16, 1024), make_sdesc(smem0 + S::kT1 + off, 16, 1024), idesc, 1u);
+          const uint32_t off = (kk >> 2) * kConvInBox + (kk & 3) * 32;
+          const uint32_t toff = (kk >> 2) * kConvBox + (kk & 3) * 32;
+          umma_ss(d, make_sdesc(prev + off, 16, 1024), make_sdesc(smem0 + S::kT1 + toff, 16, 1024), idesc, 1u);
         }
         umma_commit(&empty[s]);
         umma_commit(&tfull[a]);
@@ -263,28 +272,36 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     const int m = 32 * q + lane;                 // accumulator row = block within the tile
     uint8_t* out = smem + S::kOut;
 
-    // Toeplitz pair of channel ch: row i = et of T0 and of T1 (the columns T1 keeps)
-    auto build = [&](int ch) {
-      named_bar_sync(2, 128);                    // the previous filter is no longer read
+    // Toeplitz pair of a channel.  With the reversed filter r[u] = f(255 - u) (f = h padded
+    // with zeros), a row chunk T0[i, j0..j0+7] is r[255 - i + j0 ..] and T1[i, j0..j0+7] is
+    // r[127 - i + j0 ..]: 8 consecutive entries, copied as one 16-byte vector from the one of
+    // 8 shifted copies (rev[s][v] = r[v + s]) in which the run starts 16-byte aligned.  The
+    // copies of the next row's channel are prepared in the second buffer while the current
+    // row's tiles run, so a channel change costs only the 16-byte copies into T0 and T1.
+    auto prep = [&](int row, int rb) {            // filter of `row`'s channel -> rev buffer rb
+      named_bar_sync(2, 128);                    // filt and rev[rb] are no longer read
+      const int ch = row % p.D;
       for (int k = et; k < 256; k += 128)
         filt[k] = k < p.lh ? __bfloat16_as_ushort(p.h[static_cast<long long>(ch) * p.h_sd + k]) : 0;
       named_bar_sync(2, 128);
+      uint16_t* rv = rev + rb * 8 * kRevLen;
+      for (int idx = et; idx < 8 * kRevLen; idx += 128) {
+        const int sh = idx / kRevLen, v = idx - sh * kRevLen;
+        const int k = 255 - (v + sh);
+        rv[idx] = k >= 0 ? filt[k] : 0;
+      }
+    };
+    auto build = [&](int rb) {                   // T0, T1 from rev buffer rb
+      named_bar_sync(2, 128);                    // rev[rb] complete
+      const uint16_t* rv = rev + rb * 8 * kRevLen;
       const int i = et;
-#pragma unroll 1
+#pragma unroll 4
       for (int col = 0; col < 128; col += 8) {
-        uint32_t w0[4], w1[4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const int j = col + e;
-          const uint32_t a0 = (i - j >= 0) ? filt[i - j] : 0u;            // i - j <= 127
-          const uint32_t a1 = (i - j - 1 >= 0) ? filt[i - j - 1] : 0u;
-          w0[e >> 1] = a0 | (a1 << 16);
-          w1[e >> 1] = static_cast<uint32_t>(filt[i - j + 128]) | (static_cast<uint32_t>(filt[i - j + 127]) << 16);
-        }
-        *reinterpret_cast<uint4*>(smem + S::kT0 + sw128_off(i, col)) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-        if (col >= (2 - NPREV) * 64)
-          *reinterpret_cast<uint4*>(smem + S::kT1 + sw128_off(i, col - (2 - NPREV) * 64)) =
-              make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        const int u0 = 255 - i + col, u1 = 127 - i + col;
+        *reinterpret_cast<uint4*>(smem + S::kT0 + sw128_off(i, col)) =
+            *reinterpret_cast<const uint4*>(rv + (u0 & 7) * kRevLen + (u0 & ~7));
+        *reinterpret_cast<uint4*>(smem + S::kT1 + sw128_off(i, col)) =
+            *reinterpret_cast<const uint4*>(rv + (u1 & 7) * kRevLen + (u1 & ~7));
       }
       fence_proxy_async_smem();                  // generic writes -> tensor-core reads
       named_bar_sync(2, 128);
@@ -292,7 +309,11 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     };
 
     auto row_of = [&](int i) { return static_cast<int>((t_begin + i) / p.tiles_per_row); };
-    build(row_of(0) % p.D);
+    const int row_last = row_of(n_local - 1);
+    int rb = 0;
+    prep(row_of(0), 0);
+    build(0);
+    if (row_of(0) < row_last) prep(row_of(0) + 1, 1);
     for (int i = 0; i < n_local; ++i) {
       const int a = i & 1;
       // every epilogue thread polls; the AND over the 128 keeps their control flow uniform
@@ -301,22 +322,27 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       if (!named_bar_and(3, 128, landed)) break;
       tc_fence_after();
       const int row = row_of(i);
-      // the MMAs of tile i were the last readers of this channel's Toeplitz pair
-      if (i + 1 < n_local && row_of(i + 1) != row) build(row_of(i + 1) % p.D);
-      // accumulator row m -> 128 fp32 outputs of block m0 + m
-      uint32_t v[64];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + a * 128 + c * 32 + ((32u * q) << 16), r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          v[c * 16 + (e >> 1)] = pack_bf16x2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+      // the MMAs of tile i were the last readers of this channel's Toeplitz pair; the next
+      // row (row + 1: a CTA's tiles are consecutive) has its copies ready in the other buffer
+      const bool row_ends = i + 1 < n_local && row_of(i + 1) != row;
+      if (row_ends) {
+        rb ^= 1;
+        build(rb);
       }
+      // accumulator row m -> 128 fp32 outputs of block m0 + m (four loads, one wait)
+      uint32_t r[128];
+      const uint32_t tl = tmem_base + a * 128 + ((32u * q) << 16);
+      tmem_ld32(tl, *reinterpret_cast<uint32_t(*)[32]>(r));
+      tmem_ld32(tl + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+      tmem_ld32(tl + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
+      tmem_ld32(tl + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[a]);
+      uint32_t v[64];
+#pragma unroll
+      for (int e = 0; e < 128; e += 2) v[e >> 1] = pack_bf16x2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
       // staging: the previous tile's store has finished reading it
       if (et == 0) bulk_wait_read_all();
       named_bar_sync(2, 128);
@@ -334,6 +360,8 @@ __global__ void __launch_bounds__(kConvThreads, 1)
         tma_store_4d(&tm_y, out + kConvBox, 64, m0, ch, b);
         bulk_commit_group();
       }
+      // off the MMA's path: the copies of the row after next into the freed buffer
+      if (row_ends && row + 2 <= row_last) prep(row + 2, rb ^ 1);
     }
     if (et == 0) bulk_wait_all();
   }
@@ -380,9 +408,7 @@ __global__ void __launch_bounds__(kEdgeThreads) fir_edge_kernel(const FirEdgePar
   p.y[b * p.y_sb + ch * p.y_sd + t] = __float2bfloat16_rn(acc);
 }
 
-// Dynamic shared memory of fir_tc_kernel<NPREV>: 1 KB alignment slack + the plan above.
-__host__ __device__ constexpr size_t fir_smem_bytes(int nprev) {
-  return 1024 + (nprev == 1 ? ConvSmem<1>::kBytes : ConvSmem<2>::kBytes);
-}
+// Dynamic shared memory of fir_tc_kernel: 1 KB alignment slack + the plan above.
+__host__ __device__ constexpr size_t fir_smem_bytes() { return 1024 + ConvSmem::kBytes; }
 
 }  // namespace cpattn

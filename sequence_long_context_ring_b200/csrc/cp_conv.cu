@@ -97,13 +97,15 @@ cp_status_t run_conv(const cp_conv_plan_t* plan, const cp_tensor_t* x, const cp_
   const int64_t nblk = len / 128;
   if (nblk > 0) {
     CUtensorMap mx, my;
-    CV_TRY(make_map_bhld(&mx, x->data, c.B, c.D, nblk, 128, x->stride[0], x->stride[1], 128));
+    // input boxes of 136 blocks: a tile's 128 and the 8 before it
+    CV_TRY(make_map_bhld(&mx, x->data, c.B, c.D, nblk, 128, x->stride[0], x->stride[1], 128, 128 + kConvLead));
     CV_TRY(make_map_bhld(&my, y->data, c.B, c.D, nblk, 128, y->stride[0], y->stride[1], 128));
     ConvParams p{};
     p.D = c.D;
     p.tiles_per_row = static_cast<int>((nblk + 127) / 128);
     p.n_tiles = static_cast<long long>(c.B) * c.D * p.tiles_per_row;
     p.lh = c.lh;
+    p.kk1 = (129 - c.lh) / 16;
     p.h = static_cast<const __nv_bfloat16*>(h->data);
     p.h_sd = h->stride[0];
     p.status = status;
@@ -111,19 +113,10 @@ cp_status_t run_conv(const cp_conv_plan_t* plan, const cp_tensor_t* x, const cp_
     const int sms = sm_count();
     if (sms <= 0) return CP_ERR_CUDA;
     const long long grid = p.n_tiles < sms ? p.n_tiles : sms;
-    const int nprev = c.lh <= 65 ? 1 : 2;
-    const size_t smem = fir_smem_bytes(nprev);
-    if (nprev == 1) {
-      if (cudaFuncSetAttribute(fir_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-        return CP_ERR_CUDA;
-      fir_tc_kernel<1><<<(unsigned)grid, kConvThreads, smem, stream>>>(mx, my, p);
-    } else {
-      if (cudaFuncSetAttribute(fir_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-        return CP_ERR_CUDA;
-      fir_tc_kernel<2><<<(unsigned)grid, kConvThreads, smem, stream>>>(mx, my, p);
-    }
+    const size_t smem = fir_smem_bytes();
+    if (cudaFuncSetAttribute(fir_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return CP_ERR_CUDA;
+    fir_tc_kernel<<<(unsigned)grid, kConvThreads, smem, stream>>>(mx, my, p);
     if (cudaGetLastError() != cudaSuccess) return CP_ERR_CUDA;
   }
   const bool with_halo = halo != nullptr && c.lh > 1;

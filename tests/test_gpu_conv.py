@@ -45,6 +45,7 @@ def _ref(x, h):
     (1, 4, 128 * 130, 66, 8),          # the shortest that needs both
     (1, 2, 128 * 40, 129, 40),         # the longest filter: halo = a whole shard of 128
     (2, 80, 128 * 129, 33, 3),         # 320 tiles on 148 CTAs: channel changes inside a CTA
+    (1, 70, 128 * 300, 128, 4),        # 210 tiles: CTA ranges that start inside a row
     (1, 3, 104, 9, 2),                 # shorter than one block: the direct kernel alone
     (3, 2, 1024, 1, 4),                # one tap: no halo
 ])

@@ -114,3 +114,38 @@ def test_workspace_sizes():
     # sequence-major backward: D plus head-major copies of q, dO (Hq) and k, v, dk, dv (Hkv)
     n = 32 * 131072 * 128 * 2
     assert p.workspace_size(True) == 32 * 131072 * 4 + 2 * n + 4 * n
+
+
+# ---- the point-to-point FIR convolution (include/cp_conv.h) --------------------------------
+@pytest.mark.parametrize("kw", [
+    dict(lh=0), dict(lh=130),                  # taps outside 1..129
+    dict(L=1000, n_cp=3),                      # L % n_cp != 0
+    dict(L=64, n_cp=4, lh=18),                 # halo of 17 > shard of 16
+    dict(B=0), dict(D=0), dict(n_cp=0),
+])
+def test_conv_plan_validation_errors(kw):
+    args = dict(B=1, D=4, L=1024, lh=7, n_cp=4)
+    args.update(kw)
+    with pytest.raises(CpError) as e:
+        binding.ConvPlan(**args)
+    assert e.value.status == binding.CP_ERR_INVALID_ARG
+
+
+def test_conv_plan_accepts_the_longest_halo_and_reports_its_cost():
+    p = binding.ConvPlan(1, 4, 512, 129, 4)    # l_h - 1 = 128 = the shard length
+    nbytes, fmas = p.cost()
+    assert nbytes == 2 * 2 * 4 * 512 + 2 * 4 * 129
+    # sum over t < 512 of min(t + 1, 129), per channel
+    assert fmas == 4 * sum(min(t + 1, 129) for t in range(512))
+    p7 = binding.ConvPlan(2, 3, 40, 7, 2)
+    assert p7.cost()[1] == 2 * 3 * sum(min(t + 1, 7) for t in range(40))
+
+
+def test_conv_calls_reject_bad_arguments_before_any_launch():
+    # argument checks run on the host: null tensors and a missing plan fail without a GPU
+    lib = binding.lib()
+    assert lib.cp_conv_fir_fwd(None, None, None, None, None) == binding.CP_ERR_INVALID_ARG
+    p = binding.ConvPlan(1, 2, 256, 5, 2)
+    assert lib.cp_conv_fir_fwd(p._h, None, None, None, None) == binding.CP_ERR_INVALID_ARG
+    assert lib.cp_conv_fir_shard(p._h, 2, None, None, None, None, None) == binding.CP_ERR_INVALID_ARG
+    assert lib.cp_conv_device_status(None, None, None) == binding.CP_ERR_INVALID_ARG
