@@ -15,7 +15,8 @@ Sources (web pages on long-context sequence parallelism):
     (head x context grid), "LLMのアーキテクチャを理解する" (GQA), "スケーラビリティとメモリ管理"
     (recompute instead of store).
   * "05. 長系列の分散学習（Context Parallelism）" §3 (Hyena 演算子をどう分散するか): the
-    point-to-point FIR convolution whose shards need only the previous rank's last l_h - 1 inputs.
+    point-to-point FIR convolution whose shards need only the previous rank's last l_h - 1 inputs;
+    §4 (FFT 畳み込み): the DiF butterfly and the radix-N_cp distributed FFT convolution.
 
 Modules:
   attention  full causal softmax attention with LSE (the plain definition), row-sampled form
@@ -24,6 +25,7 @@ Modules:
   split      zig-zag / striped / contiguous rank-to-sequence maps, ring and Ulysses under them
   backward   gradient of softmax attention from its definition
   conv       causal depthwise FIR convolution and its point-to-point form with an l_h - 1 halo
+  fftconv    causal long convolution by the distributed radix-N DiF FFT (decimated spectra)
 
 Every pin of this oracle is listed in tests/test_oracle_*.py; there is no function here
 marked "parity unpinned".
@@ -35,6 +37,7 @@ from .backward import attention_backward, backward_rows_dq, backward_rows_dkdv
 from .split import (rank_positions, rank_order, shards_of_rank, step_pairs, ring_step_split,
                     ring_attention_split, seq2head_split, head2seq_split, ulysses_attention_split)
 from .conv import fir_conv, fir_conv_shard, fir_conv_cp
+from .fftconv import causal_conv, fft_conv_distributed
 
 __all__ = [
     "attention_full", "attention_rows", "forward_flops",
@@ -43,5 +46,5 @@ __all__ = [
     "attention_backward", "backward_rows_dq", "backward_rows_dkdv",
     "rank_positions", "rank_order", "shards_of_rank", "step_pairs", "ring_step_split",
     "ring_attention_split", "seq2head_split", "head2seq_split", "ulysses_attention_split",
-    "fir_conv", "fir_conv_shard", "fir_conv_cp",
+    "fir_conv", "fir_conv_shard", "fir_conv_cp", "causal_conv", "fft_conv_distributed",
 ]
