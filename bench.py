@@ -250,14 +250,15 @@ def measure_rows(dev, peaks, l_div: int = 1, only=None):
     """Device time of every other step of the hot path at its workload's shape (random bf16
     device inputs; no host data): the Ulysses permutes and the Ulysses forward (c4 shape), the
     2D forward and backward (c5 shape), the ring backward (c2 shape), one step-wise ring
-    step plus its LSE merge (c2 shape), and the point-to-point FIR convolution with a short
-    and a medium filter (c3's sequence and chunking, 4096 channels).  Each entry carries its
+    step plus its LSE merge (c2 shape), the point-to-point FIR convolution with a short and a
+    medium filter (c3's sequence and chunking, 4096 channels), and the distributed FFT
+    convolution with a sequence-long filter (c4's sequence, 4096 channels).  Each entry carries its
     roofline: HBM-bound steps against the measured copy bandwidth, contractions against the
     measured bf16 peak.  `only`: a set of row names to measure (None: all)."""
     import torch
     from sequence_long_context_ring_b200 import binding
-    from sequence_long_context_ring_b200.binding import ConvPlan, Plan
-    from sequence_long_context_ring_b200.configs import CONV_WORKLOADS, WORKLOADS
+    from sequence_long_context_ring_b200.binding import ConvPlan, FftConvPlan, Plan
+    from sequence_long_context_ring_b200.configs import CONV_WORKLOADS, FFT_WORKLOADS, WORKLOADS
 
     hbm = float(peaks["hbm_gbs"])
     tc = float(peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained")))
@@ -282,7 +283,8 @@ def measure_rows(dev, peaks, l_div: int = 1, only=None):
                                    "flops": flops}}
 
     groups = {"ulysses": ("seq2head", "head2seq", "seq2head_zigzag", "ulysses_fwd"), "2d": ("2d_fwd", "2d_bwd"),
-              "ring": ("ring_bwd", "ring_step", "ring_step_zigzag", "lse_merge"), "fir": ("fir_short", "fir_medium")}
+              "ring": ("ring_bwd", "ring_step", "ring_step_zigzag", "lse_merge"), "fir": ("fir_short", "fir_medium"),
+              "fft": ("fft_long",)}
     want = lambda grp: only is None or any(n in only for n in groups[grp])
 
     if want("ulysses"):
@@ -374,6 +376,20 @@ def measure_rows(dev, peaks, l_div: int = 1, only=None):
             if st != 0:
                 raise RuntimeError(f"device status {st} ({word:#x}) in the {key} row")
             del x, h, y, cplan
+
+    if want("fft"):
+        # distributed FFT convolution with a filter as long as the sequence (all 16 virtual
+        # ranks): filter spectra, signal slices, cross-rank inverse; bytes of its three passes
+        w = FFT_WORKLOADS["fft_long"]
+        L = w.L // l_div
+        x = rnd(w.B, w.D, L)
+        h = (rnd(w.D, L).float() * L ** -0.5).to(torch.bfloat16)
+        y = torch.empty_like(x)
+        fplan = FftConvPlan(w.B, w.D, L, w.n_cp)
+        fws = fplan.workspace(dev)
+        hbm_row("fft_long", f"[1,{w.D},{L}] bf16, filter length {L}, N_cp={w.n_cp}",
+                _time_ms(lambda: fplan.fwd(x, h, y, fws, stream), stream, reps=5), fplan.cost()[0])
+        del x, h, y, fws, fplan
     return rows
 
 

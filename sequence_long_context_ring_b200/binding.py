@@ -1,6 +1,6 @@
 """ctypes binding of libcpattn.so (argument marshalling only: every step runs in the CUDA kernels).
 
-Names follow the C ABI in include/cp_attn.h and include/cp_conv.h.  torch tensors are passed as strided views
+Names follow the C ABI in include/cp_attn.h, include/cp_conv.h and include/cp_fftconv.h.  torch tensors are passed as strided views
 (data pointer, shape, strides in elements); streams default to torch's current stream.
 There is no fallback: if the library is missing or a call fails, an exception is raised.
 """
@@ -46,13 +46,18 @@ class ConvConfig(ctypes.Structure):
                 ("n_cp", ctypes.c_int), ("wait_limit_ns", ctypes.c_uint64)]
 
 
+class FftConvConfig(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("D", ctypes.c_int), ("L", ctypes.c_int), ("n_cp", ctypes.c_int)]
+
+
 EXPORTS = [
     "cp_attn_plan", "cp_attn_plan_destroy", "cp_attn_workspace_size", "cp_attn_fwd", "cp_attn_bwd",
     "cp_layout_seq2head", "cp_layout_head2seq", "cp_ring_step", "cp_lse_merge", "cp_device_status",
     "cp_status_string", "cp_plan_step_chunk", "cp_plan_flops", "cp_plan_num_work_items", "cp_version",
     "cp_attn_fwd_noalloc", "cp_layout_seq2head_split", "cp_layout_head2seq_split",
     "cp_conv_plan", "cp_conv_plan_destroy", "cp_conv_fir_fwd", "cp_conv_fir_shard", "cp_conv_device_status",
-    "cp_conv_cost",
+    "cp_conv_cost", "cp_fftconv_plan", "cp_fftconv_plan_destroy", "cp_fftconv_workspace_size", "cp_fftconv_fwd",
+    "cp_fftconv_cost",
 ]
 
 
@@ -90,6 +95,11 @@ def lib() -> ctypes.CDLL:
             "cp_conv_fir_shard": ([P, ctypes.c_int, T, T, T, T, P], ctypes.c_int),
             "cp_conv_device_status": ([P, P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
             "cp_conv_cost": ([P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)], ctypes.c_int),
+            "cp_fftconv_plan": ([ctypes.POINTER(FftConvConfig), ctypes.POINTER(ctypes.c_void_p)], ctypes.c_int),
+            "cp_fftconv_plan_destroy": ([P], None),
+            "cp_fftconv_workspace_size": ([P, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+            "cp_fftconv_fwd": ([P, T, T, T, P, ctypes.c_size_t, P], ctypes.c_int),
+            "cp_fftconv_cost": ([P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -313,3 +323,43 @@ class ConvPlan:
         detail = ctypes.c_int()
         st = lib().cp_conv_device_status(self._h, _stream(stream), ctypes.byref(detail))
         return st, detail.value
+
+
+class FftConvPlan:
+    """A cp_fftconv plan: the causal convolution with a filter as long as the sequence by the
+    distributed radix-2N DiF FFT over n_cp contiguous virtual ranks (include/cp_fftconv.h)."""
+
+    def __init__(self, B: int, D: int, L: int, n_cp: int = 1):
+        self.cfg = FftConvConfig(B, D, L, n_cp)
+        h = ctypes.c_void_p()
+        _check(lib().cp_fftconv_plan(ctypes.byref(self.cfg), ctypes.byref(h)), "cp_fftconv_plan")
+        self._h = h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.cp_fftconv_plan_destroy(h)
+            self._h = None
+
+    def workspace_size(self) -> int:
+        n = ctypes.c_size_t()
+        _check(lib().cp_fftconv_workspace_size(self._h, ctypes.byref(n)), "cp_fftconv_workspace_size")
+        return n.value
+
+    def workspace(self, device=None) -> torch.Tensor:
+        return torch.empty(self.workspace_size(), dtype=torch.uint8, device=device or "cuda")
+
+    def cost(self):
+        """(HBM bytes, flops) of one convolution."""
+        b, f = ctypes.c_double(), ctypes.c_double()
+        _check(lib().cp_fftconv_cost(self._h, ctypes.byref(b), ctypes.byref(f)), "cp_fftconv_cost")
+        return b.value, f.value
+
+    def fwd(self, x, h, y=None, ws=None, stream=None):
+        """y = x * h, x [B, D, L], h [D, L] (bf16)."""
+        y = torch.empty_like(x) if y is None else y
+        ws = self.workspace(x.device) if ws is None else ws
+        td = [tensor_desc(t) for t in (x, h, y)]
+        _check(lib().cp_fftconv_fwd(self._h, *[ctypes.byref(t) for t in td], ws.data_ptr(), ws.numel(),
+                                    _stream(stream)), "cp_fftconv_fwd")
+        return y

@@ -8,7 +8,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libcpattn.so")
-SOURCES = [os.path.join(PKG, "csrc", "cp_attn.cu"), os.path.join(PKG, "csrc", "cp_conv.cu")]
+SOURCES = [os.path.join(PKG, "csrc", f) for f in ("cp_attn.cu", "cp_conv.cu", "cp_fftconv.cu")]
 DEPS = SOURCES + [os.path.join(PKG, "csrc", f) for f in os.listdir(os.path.join(PKG, "csrc"))] + [
     os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))]
 

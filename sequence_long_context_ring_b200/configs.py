@@ -12,6 +12,10 @@ sequence and chunking at the Llama-3-8B width (D = 4096 channels):
   fir_short   l_h = 7 taps    (a short explicit filter: halo of 6 samples per rank)
   fir_medium  l_h = 128 taps  (a medium filter: halo of 127 samples per rank)
 Inputs: x ~ N(0, 1), h ~ N(0, 1/l_h), both rounded to bf16.
+
+Distributed FFT convolution ("05. 長系列の分散学習（Context Parallelism）" §4), a long filter
+(Hyena-LI: as long as the sequence) on c4's 128K sequence at the Llama-3-8B width:
+  fft_long    D = 4096, L = 131072, N_cp = 16 (shards of 8192); h ~ N(0, 1/L)
 """
 from __future__ import annotations
 
@@ -82,4 +86,29 @@ class ConvWorkload:
 CONV_WORKLOADS = {
     "fir_short": ConvWorkload("fir_short_D4096_L212992_N16_lh7", 6, 1, 4096, 212992, 7, 16),
     "fir_medium": ConvWorkload("fir_medium_D4096_L212992_N16_lh128", 7, 1, 4096, 212992, 128, 16),
+}
+
+
+@dataclass(frozen=True)
+class FftConvWorkload:
+    name: str
+    cfg_id: int
+    B: int
+    D: int
+    L: int
+    n_cp: int
+
+    def x_shape(self):
+        return (self.B, self.D, self.L)
+
+    def h_shape(self):
+        return (self.D, self.L)
+
+    @property
+    def h_scale(self) -> float:
+        return self.L ** -0.5
+
+
+FFT_WORKLOADS = {
+    "fft_long": FftConvWorkload("fft_long_D4096_L131072_N16", 8, 1, 4096, 131072, 16),
 }

@@ -149,3 +149,33 @@ def test_conv_calls_reject_bad_arguments_before_any_launch():
     assert lib.cp_conv_fir_fwd(p._h, None, None, None, None) == binding.CP_ERR_INVALID_ARG
     assert lib.cp_conv_fir_shard(p._h, 2, None, None, None, None, None) == binding.CP_ERR_INVALID_ARG
     assert lib.cp_conv_device_status(None, None, None) == binding.CP_ERR_INVALID_ARG
+
+
+# ---- the distributed FFT convolution (include/cp_fftconv.h) --------------------------------
+@pytest.mark.parametrize("kw,err", [
+    (dict(L=1000, n_cp=3), binding.CP_ERR_INVALID_ARG),        # L % n_cp != 0
+    (dict(L=3 * 512, n_cp=3), binding.CP_ERR_UNSUPPORTED),     # n_cp not a power of two
+    (dict(L=64 * 1000, n_cp=64), binding.CP_ERR_UNSUPPORTED),  # more than 32 ranks
+    (dict(L=4 * 1000, n_cp=4), binding.CP_ERR_UNSUPPORTED),    # shard not a power of two
+    (dict(L=4 * 16384, n_cp=4), binding.CP_ERR_UNSUPPORTED),   # shard above 8192
+    (dict(L=4 * 2, n_cp=4), binding.CP_ERR_UNSUPPORTED),       # shard below 4
+    (dict(B=0), binding.CP_ERR_INVALID_ARG),
+])
+def test_fftconv_plan_validation(kw, err):
+    args = dict(B=1, D=2, L=1024, n_cp=4)
+    args.update(kw)
+    with pytest.raises(CpError) as e:
+        binding.FftConvPlan(**args)
+    assert e.value.status == err
+
+
+def test_fftconv_workspace_and_cost():
+    p = binding.FftConvPlan(2, 3, 1024, 4)
+    tw = 16 * 1024 + ((8 * 256 // 2 + 8 + 255) // 256) * 256      # w_2L^m, then w_c^m (c = 256)
+    assert p.workspace_size() == 16 * 3 * 1024 + 16 * 2 * 3 * 1024 + tw
+    nbytes, flops = p.cost()
+    D, L, B = 3, 1024, 2
+    assert nbytes == 18 * D * L + B * (34 * D * L) + B * 18 * D * L
+    assert flops > 0
+    lib = binding.lib()
+    assert lib.cp_fftconv_fwd(p._h, None, None, None, None, 0, None) == binding.CP_ERR_INVALID_ARG
