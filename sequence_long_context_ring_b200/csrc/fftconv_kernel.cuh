@@ -86,19 +86,61 @@ __device__ __forceinline__ float2 rot(float2 z) {
 // strides of the passes off a single bank.
 __device__ __forceinline__ int pidx(int i) { return i + (i >> 4); }
 
-template <int T, int K>
-__device__ __forceinline__ float2 stage_twiddle(float2 base) {
-  return rot<T, K & ((1 << T) - 1)>(base);
+// The twiddle of stage t (span s 2^t) for group element k: w_2hs^(j0 + s m) = base * w_(2^(t+1))^m,
+// m = k mod 2^t, base = w_2hs^j0 (one table read per stage).
+template <int T>
+__device__ __forceinline__ float2 stage_tf(float2 base, int k) {
+  if (T == 0) return base;
+  if (T == 1) return (k & 1) ? rot<1, 1>(base) : base;
+  const int m = k & 3;
+  return m == 0 ? base : m == 1 ? rot<2, 1>(base) : m == 2 ? rot<2, 2>(base) : rot<2, 3>(base);
 }
 
-// One pass of R (<= 3) decimation-in-frequency radix-2 stages over spans s*2^(R-1), ..., s
-// (largest first).  Group g holds the 2^R elements i0 + k s, i0 = (g / s) s 2^R + (g mod s).
-// In the stage of span hs = s 2^t the pair (k, k + 2^t) takes w_2hs^(j0 + s m), m = k mod 2^t,
-// = w_2hs^j0 * w_(2^(t+1))^m: one table read per stage, times an exact root.
 template <int R>
-__device__ __forceinline__ void dif_pass(float2* a, const float2* tw, int logc, int logs) {
-  const int c = 1 << logc, s = 1 << logs;
+__device__ __forceinline__ void dif_stages(float2 (&v)[1 << R], const float2* tw, int logc, int logs, int j0) {
+#pragma unroll
+  for (int t = R - 1; t >= 0; --t) {
+    const float2 base = tw[j0 << (logc - logs - t - 1)];   // w_c^(j0 c / (2 s 2^t))
+#pragma unroll
+    for (int k = 0; k < (1 << R); ++k) {
+      if (k & (1 << t)) continue;
+      const float2 tf = t == 0 ? stage_tf<0>(base, k) : t == 1 ? stage_tf<1>(base, k) : stage_tf<2>(base, k);
+      const float2 u = v[k], w = v[k + (1 << t)];
+      v[k] = cadd(u, w);
+      v[k + (1 << t)] = cmul(csub(u, w), tf);
+    }
+  }
+}
+
+// The mirror: decimation-in-time stages with conjugate twiddles, each the inverse of the DiF
+// butterfly times 2: (X, Y) -> (X + Y conj(w), X - Y conj(w)).
+template <int R>
+__device__ __forceinline__ void dit_stages(float2 (&v)[1 << R], const float2* tw, int logc, int logs, int j0) {
+#pragma unroll
+  for (int t = 0; t < R; ++t) {
+    const float2 base = tw[j0 << (logc - logs - t - 1)];
+#pragma unroll
+    for (int k = 0; k < (1 << R); ++k) {
+      if (k & (1 << t)) continue;
+      const float2 tf = t == 0 ? stage_tf<0>(base, k) : t == 1 ? stage_tf<1>(base, k) : stage_tf<2>(base, k);
+      const float2 u = v[k], w = cmul_conj(v[k + (1 << t)], tf);
+      v[k] = cadd(u, w);
+      v[k + (1 << t)] = csub(u, w);
+    }
+  }
+}
+
+// A pass of R radix-2 stages over spans s 2^(R-1) .. s (s = 2^logs).  Group g holds the 2^R
+// elements i0 + k s, i0 = (g - j0) 2^R + j0, j0 = g mod s.  KIND: 0 DiF in shared memory;
+// 1 DiT in shared memory; 2 DiF whose result goes to global `out` (the filter's spectrum, last
+// pass); 3 the middle of the signal's transform (s = 1): the last DiF pass, the spectral
+// product with `hq`, and the first DiT pass, in registers; 4 DiT whose result, times the
+// conjugate twiddle w_2L^(-n q) = conj(lo[n mod C1] hi[n / C1]), goes to global `out`.
+template <int R, int KIND>
+__device__ __forceinline__ void fft_pass(float2* a, const float2* tw, int logc, int logs, float2* out,
+                                         const float2* hq, const float2* lo, const float2* hi, int logc1) {
   constexpr int E = 1 << R;
+  const int c = 1 << logc, s = 1 << logs;
   const int groups = c >> R;
   for (int g = threadIdx.x; g < groups; g += kFftThreads) {
     const int j0 = g & (s - 1);
@@ -106,57 +148,36 @@ __device__ __forceinline__ void dif_pass(float2* a, const float2* tw, int logc, 
     float2 v[E];
 #pragma unroll
     for (int k = 0; k < E; ++k) v[k] = a[pidx(i0 + k * s)];
+    if (KIND == 0 || KIND == 2 || KIND == 3) dif_stages<R>(v, tw, logc, logs, j0);
+    if (KIND == 3) {
+      // s = 1: the group's elements are contiguous in the spectrum's storage order
 #pragma unroll
-    for (int t = R - 1; t >= 0; --t) {
-      const float2 base = tw[j0 << (logc - logs - t - 1)];   // w_c^(j0 c / (2 s 2^t))
+      for (int k = 0; k < E; ++k) v[k] = cmul(v[k], hq[i0 + k]);
+    }
+    if (KIND == 1 || KIND == 3 || KIND == 4) dit_stages<R>(v, tw, logc, logs, j0);
+    if (KIND == 2) {
+#pragma unroll
+      for (int k = 0; k < E; ++k) out[i0 + k * s] = v[k];
+    } else if (KIND == 4) {
+      const int m1 = (1 << logc1) - 1;
 #pragma unroll
       for (int k = 0; k < E; ++k) {
-        if (k & (1 << t)) continue;
-        const float2 u = v[k], w = v[k + (1 << t)];
-        float2 tf;
-        if (t == 0) tf = base;
-        else if (t == 1) tf = (k & 1) ? rot<1, 1>(base) : base;
-        else tf = (k & 3) == 0 ? base : (k & 3) == 1 ? rot<2, 1>(base) : (k & 3) == 2 ? rot<2, 2>(base) : rot<2, 3>(base);
-        v[k] = cadd(u, w);
-        v[k + (1 << t)] = cmul(csub(u, w), tf);
+        const int n = i0 + k * s;
+        out[n] = cmul_conj(v[k], cmul(lo[n & m1], hi[n >> logc1]));
       }
-    }
+    } else {
 #pragma unroll
-    for (int k = 0; k < E; ++k) a[pidx(i0 + k * s)] = v[k];
+      for (int k = 0; k < E; ++k) a[pidx(i0 + k * s)] = v[k];
+    }
   }
 }
 
-// The mirror: decimation-in-time stages of spans s, ..., s*2^(R-1) with conjugate twiddles,
-// each the inverse of the DiF butterfly times 2: (X, Y) -> (X + Y conj(w), X - Y conj(w)).
-template <int R>
-__device__ __forceinline__ void dit_pass(float2* a, const float2* tw, int logc, int logs) {
-  const int c = 1 << logc, s = 1 << logs;
-  constexpr int E = 1 << R;
-  const int groups = c >> R;
-  for (int g = threadIdx.x; g < groups; g += kFftThreads) {
-    const int j0 = g & (s - 1);
-    const int i0 = (g - j0) * E + j0;
-    float2 v[E];
-#pragma unroll
-    for (int k = 0; k < E; ++k) v[k] = a[pidx(i0 + k * s)];
-#pragma unroll
-    for (int t = 0; t < R; ++t) {
-      const float2 base = tw[j0 << (logc - logs - t - 1)];   // w_c^(j0 c / (2 s 2^t))
-#pragma unroll
-      for (int k = 0; k < E; ++k) {
-        if (k & (1 << t)) continue;
-        float2 tf;
-        if (t == 0) tf = base;
-        else if (t == 1) tf = (k & 1) ? rot<1, 1>(base) : base;
-        else tf = (k & 3) == 0 ? base : (k & 3) == 1 ? rot<2, 1>(base) : (k & 3) == 2 ? rot<2, 2>(base) : rot<2, 3>(base);
-        const float2 u = v[k], w = cmul_conj(v[k + (1 << t)], tf);
-        v[k] = cadd(u, w);
-        v[k + (1 << t)] = csub(u, w);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < E; ++k) a[pidx(i0 + k * s)] = v[k];
-  }
+template <int KIND>
+__device__ __forceinline__ void run_pass(int r, float2* a, const float2* tw, int logc, int logs, float2* out,
+                                         const float2* hq, const float2* lo, const float2* hi, int logc1) {
+  if (r == 1) fft_pass<1, KIND>(a, tw, logc, logs, out, hq, lo, hi, logc1);
+  else if (r == 2) fft_pass<2, KIND>(a, tw, logc, logs, out, hq, lo, hi, logc1);
+  else fft_pass<3, KIND>(a, tw, logc, logs, out, hq, lo, hi, logc1);
 }
 
 // Split log2(c) stages into passes of at most 3 (as even as possible); forward: largest spans
@@ -171,17 +192,6 @@ __device__ __forceinline__ int fft_passes(int logc, int* radix) {
   return np;
 }
 
-__device__ __forceinline__ void run_dif(float2* a, const float2* tw, int logc, int r, int logs) {
-  if (r == 1) dif_pass<1>(a, tw, logc, logs);
-  else if (r == 2) dif_pass<2>(a, tw, logc, logs);
-  else dif_pass<3>(a, tw, logc, logs);
-}
-__device__ __forceinline__ void run_dit(float2* a, const float2* tw, int logc, int r, int logs) {
-  if (r == 1) dit_pass<1>(a, tw, logc, logs);
-  else if (r == 2) dit_pass<2>(a, tw, logc, logs);
-  else dit_pass<3>(a, tw, logc, logs);
-}
-
 // MODE 0: the filter's spectra H_q -> p.spec.  MODE 1: the signal's w_q -> p.w.
 template <int MODE>
 __global__ void __launch_bounds__(kFftThreads, 2) fftconv_slice_kernel(const FftParams p) {
@@ -190,16 +200,20 @@ __global__ void __launch_bounds__(kFftThreads, 2) fftconv_slice_kernel(const Fft
   const int row = blockIdx.x / Q;
   const int q = blockIdx.x - row * Q;
   const int c = p.c;
+  const int logc1 = p.logc < 6 ? p.logc : 6;          // n = n_lo + C1 n_hi, C1 = min(c, 64)
+  const int c1 = 1 << logc1;
   float2* a = fsm;                           // c values at pidx(i)
   float2* tw = fsm + c + c / 16;             // c / 2 twiddles w_c^m
   float2* cf = tw + c / 2;                   // N cross-rank coefficients w_2N^(r q)
-  float2* ew = cf + kFftMaxN;                // w_2L^(e q), e < 8
+  float2* lo = cf + kFftMaxN;                // w_2L^(u q), u < C1
+  float2* hi = lo + 64;                      // w_2L^(C1 v q), v < c / C1 (<= 128)
 
 #pragma unroll 8
   for (int m = threadIdx.x; m < c / 2; m += kFftThreads) tw[m] = p.twc[m];
-  // w_2N^(r q) = w_2L^((r q mod 2N) c); ew[e] = w_2L^(e q)
+  // w_2N^(r q) = w_2L^((r q mod 2N) c); lo/hi: every index below 2L (u q < C1 2N <= 2L, C1 v q < c 2N)
   for (int r = threadIdx.x; r < p.N; r += kFftThreads) cf[r] = p.tw2l[((r * q) % Q) * c];
-  if (threadIdx.x < 8) ew[threadIdx.x] = p.tw2l[(threadIdx.x * q) % (2 * p.L)];
+  if (threadIdx.x < c1) lo[threadIdx.x] = p.tw2l[threadIdx.x * q];
+  for (int v = threadIdx.x; v < (c >> logc1); v += kFftThreads) hi[v] = p.tw2l[(v << logc1) * q];
   __syncthreads();
 
   // cross-rank stage, 8 consecutive samples per thread (16-byte loads of every shard):
@@ -243,62 +257,43 @@ __global__ void __launch_bounds__(kFftThreads, 2) fftconv_slice_kernel(const Fft
         }
       }
     }
-    // w_2L^(n q) = w_2L^(n0 q) w_2L^(e q); n0 q < 2N c = 2L
-    const float2 t0 = p.tw2l[n0 * q];
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (n0 + e < c) a[pidx(n0 + e)] = cmul(acc[e], cmul(t0, ew[e]));
+    for (int e = 0; e < 8; ++e) {
+      const int n = n0 + e;
+      if (n < c) a[pidx(n)] = cmul(acc[e], cmul(lo[n & (c1 - 1)], hi[n >> logc1]));
+    }
   }
   __syncthreads();
 
   int radix[5];
   const int np = fft_passes(p.logc, radix);
+  const long long slice = (static_cast<long long>(row) * Q + q) * c;
   int logs = p.logc;
-  for (int i = 0; i < np; ++i) {
+  for (int i = 0; i + 1 < np; ++i) {
     logs -= radix[i];
-    run_dif(a, tw, p.logc, radix[i], logs);
+    run_pass<0>(radix[i], a, tw, p.logc, logs, nullptr, nullptr, nullptr, nullptr, 0);
     __syncthreads();
   }
-
-  const long long slice = (static_cast<long long>(row) * Q + q) * c;
+  // logs is now radix[np-1]: the last pass has s = 1
   if (MODE == 0) {
-    for (int k = threadIdx.x; k < c; k += kFftThreads) p.spec[slice + k] = a[pidx(k)];
+    run_pass<2>(radix[np - 1], a, tw, p.logc, 0, p.spec + slice, nullptr, nullptr, nullptr, 0);
     return;
   }
   const float2* hq = p.spec + (static_cast<long long>(ch) * Q + q) * c;
-  for (int k0 = threadIdx.x; k0 < c; k0 += 4 * kFftThreads) {
-    float2 hv[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int k = k0 + u * kFftThreads;
-      hv[u] = k < c ? hq[k] : make_float2(0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int k = k0 + u * kFftThreads;
-      if (k < c) a[pidx(k)] = cmul(a[pidx(k)], hv[u]);
-    }
-  }
+  run_pass<3>(radix[np - 1], a, tw, p.logc, 0, nullptr, hq, nullptr, nullptr, 0);
   __syncthreads();
-  logs = 0;
-  for (int i = np - 1; i >= 0; --i) {
-    run_dit(a, tw, p.logc, radix[i], logs);
+  logs = radix[np - 1];
+  for (int i = np - 2; i >= 1; --i) {
+    run_pass<1>(radix[i], a, tw, p.logc, logs, nullptr, nullptr, nullptr, nullptr, 0);
     logs += radix[i];
     __syncthreads();
   }
-  // w_q(n) = w_2L^(-n q) * (local inverse)
-  for (int m0 = threadIdx.x; m0 < c; m0 += 4 * kFftThreads) {
-    float2 tv[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int n = m0 + u * kFftThreads;
-      tv[u] = n < c ? p.tw2l[(n & ~7) * q] : make_float2(1.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int n = m0 + u * kFftThreads;
-      if (n < c) p.w[slice + n] = cmul_conj(a[pidx(n)], cmul(tv[u], ew[n & 7]));
-    }
+  if (np >= 2) {
+    // the last inverse pass writes w_q(n) = w_2L^(-n q) * (local inverse) straight to global
+    run_pass<4>(radix[0], a, tw, p.logc, logs, p.w + slice, nullptr, lo, hi, logc1);
+  } else {
+    for (int n = threadIdx.x; n < c; n += kFftThreads)
+      p.w[slice + n] = cmul_conj(a[pidx(n)], cmul(lo[n & (c1 - 1)], hi[n >> logc1]));
   }
 }
 
@@ -343,7 +338,7 @@ __global__ void __launch_bounds__(kFftThreads) fftconv_inverse_kernel(const FftI
 }
 
 __host__ __device__ constexpr size_t fftconv_smem_bytes(int c, int N) {
-  return (static_cast<size_t>(c) + c / 16 + c / 2 + kFftMaxN + 8) * sizeof(float2);
+  return (static_cast<size_t>(c) + c / 16 + c / 2 + kFftMaxN + 64 + 128) * sizeof(float2);
 }
 
 }  // namespace cpattn
