@@ -472,18 +472,29 @@ def run_ours(args, w):
                   for b in (qb, kb, vb))
     oh = torch.empty(w.q_shape(), dtype=torch.bfloat16).pin_memory()
     lh = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32).pin_memory()
-    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if w.mode == "ring":
+        # the library's host-buffer entry point: copies in and out overlap the kernels
+        hws = torch.empty(plan.host_workspace_size(), dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            plan.fwd_host(qh, kh, vh, oh, lh, hws, stream)
+    else:
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            plan.fwd(qd, kd, vd, o, lse, ws, stream)
+            oh.copy_(o, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+    e2e_step()                                   # warm-up (staging buffers touched once)
     barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.e2e_steps):
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        plan.fwd(qd, kd, vd, o, lse, ws, stream)
-        oh.copy_(o, non_blocking=True)
-        lh.copy_(lse, non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)

@@ -161,6 +161,22 @@ cp_status_t cp_attn_bwd(const cp_plan_t* plan, const cp_tensor_t* q, const cp_te
 cp_status_t cp_attn_fwd_noalloc(const cp_plan_t* plan, const cp_tensor_t* q, const cp_tensor_t* k,
                                 const cp_tensor_t* v, cp_tensor_t* o, cp_tensor_t* lse, void* stream);
 
+/* Forward of a RING plan with the tensors in HOST memory: q, k, v, o [B, H, L, d] bf16 and lse
+ * [B, Hq, L] fp32, each contiguous (canonical strides), preferably page-locked (pageable memory
+ * works but its copies do not overlap the kernels).  The library copies the inputs in, runs
+ * the same forward kernel, and copies O and LSE out, pipelined over blocks of KV heads: while
+ * one block computes on `stream`, the next block's Q/K/V arrive and the previous block's O/LSE
+ * leave on two internal streams (GQA blocks are independent problems, so the result is
+ * bit-identical to cp_attn_fwd).  Device staging for all five tensors comes from `ws`, a
+ * device buffer of at least cp_attn_host_workspace_size bytes, 256-byte aligned.  Everything
+ * is enqueued behind the work already on `stream`; the host buffers are complete, and `ws`
+ * free, when `stream` reaches the point of this call's return.  Other modes: CP_ERR_UNSUPPORTED. */
+cp_status_t cp_attn_fwd_host(const cp_plan_t* plan, const cp_tensor_t* q, const cp_tensor_t* k,
+                             const cp_tensor_t* v, cp_tensor_t* o, cp_tensor_t* lse, void* ws,
+                             size_t ws_bytes, void* stream);
+/* Device bytes cp_attn_fwd_host stages through (Q, K, V, O, LSE, each 256-byte aligned). */
+cp_status_t cp_attn_host_workspace_size(const cp_plan_t* plan, size_t* bytes);
+
 /* Ulysses all-to-all on one GPU ([CP] §2, [UL] step 2): in [B, L, H, d] (rank s holds rows
  * [s*c, (s+1)*c)) -> out [B, H, L, d] (rank r' holds heads [r'*H/N, (r'+1)*H/N) for all L):
  *     out[b, r'*H/N + h', s*c + t, :] = in[b, s*c + t, r'*H/N + h', :].

@@ -56,7 +56,7 @@ EXPORTS = [
     "cp_status_string", "cp_plan_step_chunk", "cp_plan_flops", "cp_plan_num_work_items", "cp_version",
     "cp_attn_fwd_noalloc", "cp_layout_seq2head_split", "cp_layout_head2seq_split",
     "cp_conv_plan", "cp_conv_plan_destroy", "cp_conv_fir_fwd", "cp_conv_fir_shard", "cp_conv_device_status",
-    "cp_conv_cost", "cp_fftconv_plan", "cp_fftconv_plan_destroy", "cp_fftconv_workspace_size", "cp_fftconv_fwd",
+    "cp_conv_cost", "cp_attn_fwd_host", "cp_attn_host_workspace_size", "cp_fftconv_plan", "cp_fftconv_plan_destroy", "cp_fftconv_workspace_size", "cp_fftconv_fwd",
     "cp_fftconv_cost",
 ]
 
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
             "cp_attn_fwd_noalloc": ([P, T, T, T, T, T, P], ctypes.c_int),
             "cp_layout_seq2head_split": ([ctypes.c_int, ctypes.c_int, T, T, P], ctypes.c_int),
             "cp_layout_head2seq_split": ([ctypes.c_int, ctypes.c_int, T, T, P], ctypes.c_int),
+            "cp_attn_fwd_host": ([P, T, T, T, T, T, P, ctypes.c_size_t, P], ctypes.c_int),
+            "cp_attn_host_workspace_size": ([P, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "cp_conv_plan": ([ctypes.POINTER(ConvConfig), ctypes.POINTER(ctypes.c_void_p)], ctypes.c_int),
             "cp_conv_plan_destroy": ([P], None),
             "cp_conv_fir_fwd": ([P, T, T, T, P], ctypes.c_int),
@@ -201,6 +203,22 @@ class Plan:
         td = [tensor_desc(t) for t in (q, k, v, o, lse)]
         _check(lib().cp_attn_fwd(self._h, *[ctypes.byref(t) for t in td], wptr, wlen, _stream(stream)),
                "cp_attn_fwd")
+        return o, lse
+
+    def host_workspace_size(self) -> int:
+        n = ctypes.c_size_t()
+        _check(lib().cp_attn_host_workspace_size(self._h, ctypes.byref(n)), "cp_attn_host_workspace_size")
+        return n.value
+
+    def fwd_host(self, q, k, v, o, lse, ws=None, stream=None):
+        """Forward of a ring plan on HOST tensors (contiguous, preferably pinned): the library
+        copies in, computes and copies out, overlapping the transfers with the kernels.  ws:
+        device staging of host_workspace_size() bytes."""
+        if ws is None:
+            ws = torch.empty(self.host_workspace_size(), dtype=torch.uint8, device="cuda")
+        td = [tensor_desc(t) for t in (q, k, v, o, lse)]
+        _check(lib().cp_attn_fwd_host(self._h, *[ctypes.byref(t) for t in td], ws.data_ptr(), ws.numel(),
+                                      _stream(stream)), "cp_attn_fwd_host")
         return o, lse
 
     def fwd_noalloc(self, q, k, v, o, lse, stream=None):

@@ -63,12 +63,16 @@ struct DqItem {
 // Work items longest first: last chunk, last query tiles (the causal work grows with the row).
 __device__ __forceinline__ DqItem decode_dq_item(const DqParams& p) {
   DqItem it;
-  const int n_inner = p.B * p.Hq;
-  const int pos = blockIdx.x / n_inner;
-  const int inner = blockIdx.x - pos * n_inner;
-  it.b = inner / p.Hq;
-  it.h = inner - it.b * p.Hq;
-  it.g = it.h / p.G;
+  // (batch, KV head)-major: the CTAs in flight are the query tiles of one KV group's heads and
+  // stream that group's K/V tiles, re-read from L2; within it longest first
+  const int n_pos = p.n_chunks * p.tiles_per_chunk;
+  const int per_bg = n_pos * p.G;
+  const int bg = blockIdx.x / per_bg;
+  const int rem = blockIdx.x - bg * per_bg;
+  const int pos = rem / p.G;
+  it.b = bg / p.Hkv;
+  it.g = bg - it.b * p.Hkv;
+  it.h = it.g * p.G + (rem - pos * p.G);
   it.r = p.n_chunks - 1 - pos / p.tiles_per_chunk;
   const int qpos = p.tiles_per_chunk - 1 - pos % p.tiles_per_chunk;
   const int c0 = it.r * p.chunk_len;

@@ -70,11 +70,14 @@ struct BwdItem {
 
 __device__ __forceinline__ BwdItem decode_bwd_item(const BwdParams& p) {
   BwdItem it;
-  const int n_inner = p.B * p.Hkv;
-  const int pos = blockIdx.x / n_inner;        // longest first: the earliest keys see the most queries
-  const int inner = blockIdx.x - pos * n_inner;
-  it.b = inner / p.Hkv;
-  it.g = inner - it.b * p.Hkv;
+  // (batch, KV head)-major, so the CTAs in flight stream the same query / dO tiles of one
+  // KV group and re-read them from L2; within it longest first: the earliest keys see the
+  // most queries
+  const int n_pos = p.n_chunks * p.tiles_per_chunk;
+  const int bg = blockIdx.x / n_pos;
+  const int pos = blockIdx.x - bg * n_pos;
+  it.b = bg / p.Hkv;
+  it.g = bg - it.b * p.Hkv;
   it.j = pos / p.tiles_per_chunk;
   const int tt = pos - it.j * p.tiles_per_chunk;
   const int c0 = it.j * p.chunk_len;

@@ -573,6 +573,140 @@ cp_status_t cp_attn_fwd(const cp_plan_t* plan, const cp_tensor_t* q, const cp_te
   return head_buf_to_seq(oh, o, s, c.split, c.n_cp);
 }
 
+namespace {
+
+// A host tensor in canonical contiguous layout with the given shape.
+cp_status_t check_host(const cp_tensor_t* t, cp_dtype_t dt, int nd, const int64_t* shape) {
+  if (!t || !t->data || t->ndim != nd || t->dtype != dt) return CP_ERR_INVALID_ARG;
+  int64_t stride = 1;
+  for (int i = nd - 1; i >= 0; --i) {
+    if (t->shape[i] != shape[i]) return CP_ERR_INVALID_ARG;
+    if (t->stride[i] != stride) return CP_ERR_ALIGNMENT;
+    stride *= shape[i];
+  }
+  return CP_OK;
+}
+
+// KV heads per pipelined block: the largest divisor of Hkv that gives at most 8 blocks per
+// batch element (enough blocks to hide the transfers, few enough that every launch still fills
+// the GPU many times over).
+int host_block_heads(int Hkv) {
+  for (int nb = 8; nb >= 1; --nb)
+    if (Hkv % nb == 0) return Hkv / nb;
+  return Hkv;
+}
+
+}  // namespace
+
+cp_status_t cp_attn_host_workspace_size(const cp_plan_t* plan, size_t* bytes) {
+  if (!plan || !bytes) return CP_ERR_INVALID_ARG;
+  const cp_attn_config_t& c = plan->cfg;
+  const size_t nq = (size_t)c.B * c.Hq * c.L * c.d, nkv = (size_t)c.B * c.Hkv * c.L * c.d;
+  *bytes = 2 * align256(nq * 2) + 2 * align256(nkv * 2) + align256((size_t)c.B * c.Hq * c.L * 4);
+  return CP_OK;
+}
+
+cp_status_t cp_attn_fwd_host(const cp_plan_t* plan, const cp_tensor_t* q, const cp_tensor_t* k,
+                             const cp_tensor_t* v, cp_tensor_t* o, cp_tensor_t* lse, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (!plan) return CP_ERR_INVALID_ARG;
+  const cp_attn_config_t& c = plan->cfg;
+  if (c.mode != CP_MODE_RING) return CP_ERR_UNSUPPORTED;
+  const int64_t sq[4] = {c.B, c.Hq, c.L, c.d}, skv[4] = {c.B, c.Hkv, c.L, c.d}, sl[3] = {c.B, c.Hq, c.L};
+  CP_TRY(check_host(q, CP_BF16, 4, sq));
+  CP_TRY(check_host(k, CP_BF16, 4, skv));
+  CP_TRY(check_host(v, CP_BF16, 4, skv));
+  CP_TRY(check_host(o, CP_BF16, 4, sq));
+  CP_TRY(check_host(lse, CP_FP32, 3, sl));
+  size_t need = 0;
+  CP_TRY(cp_attn_host_workspace_size(plan, &need));
+  if (!ws || ws_bytes < need) return CP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return CP_ERR_ALIGNMENT;
+  const size_t nq = (size_t)c.B * c.Hq * c.L * c.d, nkv = (size_t)c.B * c.Hkv * c.L * c.d;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint8_t* dq = w;
+  w += align256(nq * 2);
+  uint8_t* dk = w;
+  w += align256(nkv * 2);
+  uint8_t* dv = w;
+  w += align256(nkv * 2);
+  uint8_t* dO = w;
+  w += align256(nq * 2);
+  float* dl = reinterpret_cast<float*>(w);
+
+  const cudaStream_t s = as_stream(stream);
+  const int hb = host_block_heads(c.Hkv);      // KV heads per block
+  const int nb = c.Hkv / hb;                   // blocks per batch element
+  const int G = plan->G;
+  const size_t q_blk = (size_t)hb * G * c.L * c.d * 2, kv_blk = (size_t)hb * c.L * c.d * 2;
+  const size_t l_blk = (size_t)hb * G * c.L * 4;
+  const int n_parts = c.B * nb;
+
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t e_start = nullptr, e_done = nullptr;
+  cp_status_t st = CP_OK;
+  auto cuda_ok = [&](cudaError_t e) {
+    if (e != cudaSuccess && st == CP_OK) st = CP_ERR_CUDA;
+    return st == CP_OK;
+  };
+  if (!cuda_ok(cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking)) ||
+      !cuda_ok(cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking)) ||
+      !cuda_ok(cudaEventCreateWithFlags(&e_start, cudaEventDisableTiming)) ||
+      !cuda_ok(cudaEventCreateWithFlags(&e_done, cudaEventDisableTiming)) || !cuda_ok(cudaEventRecord(e_start, s)) ||
+      !cuda_ok(cudaStreamWaitEvent(s_in, e_start, 0)) || !cuda_ok(cudaStreamWaitEvent(s_out, e_start, 0))) {
+  } else {
+    for (int part = 0; part < n_parts && st == CP_OK; ++part) {
+      const int b = part / nb, kb = part - b * nb;
+      const size_t qoff = ((size_t)b * c.Hq + (size_t)kb * hb * G) * c.L * c.d * 2;
+      const size_t kvoff = ((size_t)b * c.Hkv + (size_t)kb * hb) * c.L * c.d * 2;
+      const size_t loff = ((size_t)b * c.Hq + (size_t)kb * hb * G) * c.L * 4;
+      cudaEvent_t e_in = nullptr, e_comp = nullptr;
+      if (!cuda_ok(cudaEventCreateWithFlags(&e_in, cudaEventDisableTiming)) ||
+          !cuda_ok(cudaEventCreateWithFlags(&e_comp, cudaEventDisableTiming)))
+        break;
+      // 1) this block's inputs in (behind the previous block's, on s_in)
+      cuda_ok(cudaMemcpyAsync(dq + qoff, static_cast<const uint8_t*>(q->data) + qoff, q_blk, cudaMemcpyHostToDevice, s_in));
+      cuda_ok(cudaMemcpyAsync(dk + kvoff, static_cast<const uint8_t*>(k->data) + kvoff, kv_blk, cudaMemcpyHostToDevice, s_in));
+      cuda_ok(cudaMemcpyAsync(dv + kvoff, static_cast<const uint8_t*>(v->data) + kvoff, kv_blk, cudaMemcpyHostToDevice, s_in));
+      cuda_ok(cudaEventRecord(e_in, s_in));
+      cuda_ok(cudaStreamWaitEvent(s, e_in, 0));
+      // 2) the forward of the block on the caller's stream: the same kernel over the block's
+      //    heads (views offset to them; the geometry counts only the block's heads)
+      if (st == CP_OK) {
+        FwdParams p{};
+        fill_geometry(plan, c.n_cp, p);
+        p.B = 1;
+        p.Hq = hb * G;
+        p.Hkv = hb;
+        p.n_inner = p.pair_heads ? hb * (G / 2) : hb * G;
+        const int64_t grid = (int64_t)p.n_chunks * p.pos_per_chunk * p.n_inner;
+        const int64_t hsz = (int64_t)c.L * c.d;
+        FwdOut out{dO + qoff, (int64_t)hb * G * hsz, hsz, c.d, 0, reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(dl) + loff),
+                   (int64_t)hb * G * c.L, c.L, 1};
+        st = run_fwd_kernel(plan, p, contiguous_view(dq + qoff, 1, hb * G, c.L, c.d),
+                            contiguous_view(dk + kvoff, 1, hb, c.L, c.d), contiguous_view(dv + kvoff, 1, hb, c.L, c.d),
+                            out, grid, s);
+      }
+      cuda_ok(cudaEventRecord(e_comp, s));
+      // 3) its outputs out (on s_out, behind the previous block's)
+      cuda_ok(cudaStreamWaitEvent(s_out, e_comp, 0));
+      cuda_ok(cudaMemcpyAsync(static_cast<uint8_t*>(o->data) + qoff, dO + qoff, q_blk, cudaMemcpyDeviceToHost, s_out));
+      cuda_ok(cudaMemcpyAsync(static_cast<uint8_t*>(lse->data) + loff, reinterpret_cast<uint8_t*>(dl) + loff, l_blk,
+                              cudaMemcpyDeviceToHost, s_out));
+      cudaEventDestroy(e_in);   // released once recorded work completes
+      cudaEventDestroy(e_comp);
+    }
+    // the caller's stream continues only after the last block's outputs have landed
+    cuda_ok(cudaEventRecord(e_done, s_out));
+    cuda_ok(cudaStreamWaitEvent(s, e_done, 0));
+  }
+  if (e_start) cudaEventDestroy(e_start);
+  if (e_done) cudaEventDestroy(e_done);
+  if (s_in) cudaStreamDestroy(s_in);    // resources freed after the enqueued work completes
+  if (s_out) cudaStreamDestroy(s_out);
+  return st;
+}
+
 cp_status_t cp_ring_step(const cp_plan_t* plan, int rank, int step, const cp_tensor_t* q, const cp_tensor_t* k,
                          const cp_tensor_t* v, cp_tensor_t* o_part, cp_tensor_t* lse_part, void* stream) {
   if (!plan) return CP_ERR_INVALID_ARG;

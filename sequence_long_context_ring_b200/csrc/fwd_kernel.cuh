@@ -102,36 +102,43 @@ __device__ __forceinline__ int step_tiles(const FwdParams& p, int r, int n_diag,
 __device__ __forceinline__ Item decode_item(const FwdParams& p) {
   Item it;
   const int idx = blockIdx.x;
-  const int pos = idx / p.n_inner;
-  const int inner = idx - pos * p.n_inner;
-  int qpos;
+  // items of one KV head: a pair of query heads (pair_heads) or one query head (else)
+  const int ig = p.pair_heads ? (p.G >> 1) : p.G;
+  int pos, bg, w, qpos;
   if (p.step_rank >= 0) {
+    pos = idx / p.n_inner;
+    const int inner = idx - pos * p.n_inner;
+    bg = inner / ig;
+    w = inner - bg * ig;
     it.r = p.step_rank;
     qpos = p.pos_per_chunk - 1 - pos;
   } else {
-    // longest-first: last chunk, last query tiles first (the causal work grows with the row)
+    // KV-head-major: all of one (batch, KV head)'s items before the next, so the CTAs in flight
+    // walk the same K/V chunks (in ascending order) and re-read them from L2, not DRAM; within
+    // a KV head, longest first: last chunk, last query tiles first (the causal work grows with
+    // the row)
+    const int per_bg = p.n_chunks * p.pos_per_chunk * ig;
+    bg = idx / per_bg;
+    const int rem = idx - bg * per_bg;
+    pos = rem / ig;
+    w = rem - pos * ig;
     it.r = p.n_chunks - 1 - pos / p.pos_per_chunk;
     qpos = p.pos_per_chunk - 1 - pos % p.pos_per_chunk;
   }
   const int c0 = it.r * p.chunk_len;
   it.q_end = min(c0 + p.chunk_len, p.L);
   int last;  // last valid query row of the item
+  it.b = bg / p.Hkv;
+  it.g = bg - it.b * p.Hkv;
   if (p.pair_heads) {
-    const int half = p.G >> 1;
-    it.b = inner / (p.Hkv * half);
-    const int rem = inner - it.b * (p.Hkv * half);
-    it.g = rem / half;
-    const int pr = rem - it.g * half;
-    it.headA = it.g * p.G + 2 * pr;
+    it.headA = it.g * p.G + 2 * w;
     it.headB = it.headA + 1;
     it.rowA = c0 + qpos * kBM;
     it.rowB = it.rowA;
     last = min(it.rowA + kBM, it.q_end) - 1;
   } else {
-    it.b = inner / p.Hq;
-    it.headA = inner - it.b * p.Hq;
+    it.headA = it.g * p.G + w;
     it.headB = it.headA;
-    it.g = it.headA / p.G;
     it.rowA = c0 + (2 * qpos) * kBM;
     it.rowB = it.rowA + kBM;
     last = min(it.rowB + kBM, it.q_end) - 1;
