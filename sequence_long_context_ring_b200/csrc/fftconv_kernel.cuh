@@ -96,11 +96,20 @@ __device__ __forceinline__ float2 stage_tf(float2 base, int k) {
   return m == 0 ? base : m == 1 ? rot<2, 1>(base) : m == 2 ? rot<2, 2>(base) : rot<2, 3>(base);
 }
 
+// bases[t] = w_(2 s 2^t)^j0: the pass's table holds the largest-span root per j0 (consecutive
+// j0 in consecutive entries: no bank conflicts across a warp), the others are its squares.
 template <int R>
-__device__ __forceinline__ void dif_stages(float2 (&v)[1 << R], const float2* tw, int logc, int logs, int j0) {
+__device__ __forceinline__ void stage_bases(float2 (&bases)[R], const float2* tp, int j0) {
+  bases[R - 1] = tp[j0];
+#pragma unroll
+  for (int t = R - 1; t > 0; --t) bases[t - 1] = cmul(bases[t], bases[t]);
+}
+
+template <int R>
+__device__ __forceinline__ void dif_stages(float2 (&v)[1 << R], const float2 (&bases)[R]) {
 #pragma unroll
   for (int t = R - 1; t >= 0; --t) {
-    const float2 base = tw[j0 << (logc - logs - t - 1)];   // w_c^(j0 c / (2 s 2^t))
+    const float2 base = bases[t];
 #pragma unroll
     for (int k = 0; k < (1 << R); ++k) {
       if (k & (1 << t)) continue;
@@ -115,10 +124,10 @@ __device__ __forceinline__ void dif_stages(float2 (&v)[1 << R], const float2* tw
 // The mirror: decimation-in-time stages with conjugate twiddles, each the inverse of the DiF
 // butterfly times 2: (X, Y) -> (X + Y conj(w), X - Y conj(w)).
 template <int R>
-__device__ __forceinline__ void dit_stages(float2 (&v)[1 << R], const float2* tw, int logc, int logs, int j0) {
+__device__ __forceinline__ void dit_stages(float2 (&v)[1 << R], const float2 (&bases)[R]) {
 #pragma unroll
   for (int t = 0; t < R; ++t) {
-    const float2 base = tw[j0 << (logc - logs - t - 1)];
+    const float2 base = bases[t];
 #pragma unroll
     for (int k = 0; k < (1 << R); ++k) {
       if (k & (1 << t)) continue;
@@ -137,7 +146,7 @@ __device__ __forceinline__ void dit_stages(float2 (&v)[1 << R], const float2* tw
 // product with `hq`, and the first DiT pass, in registers; 4 DiT whose result, times the
 // conjugate twiddle w_2L^(-n q) = conj(lo[n mod C1] hi[n / C1]), goes to global `out`.
 template <int R, int KIND>
-__device__ __forceinline__ void fft_pass(float2* a, const float2* tw, int logc, int logs, float2* out,
+__device__ __forceinline__ void fft_pass(float2* a, const float2* tp, int logc, int logs, float2* out,
                                          const float2* hq, const float2* lo, const float2* hi, int logc1) {
   constexpr int E = 1 << R;
   const int c = 1 << logc, s = 1 << logs;
@@ -148,13 +157,15 @@ __device__ __forceinline__ void fft_pass(float2* a, const float2* tw, int logc, 
     float2 v[E];
 #pragma unroll
     for (int k = 0; k < E; ++k) v[k] = a[pidx(i0 + k * s)];
-    if (KIND == 0 || KIND == 2 || KIND == 3) dif_stages<R>(v, tw, logc, logs, j0);
+    float2 bases[R];
+    stage_bases<R>(bases, tp, j0);
+    if (KIND == 0 || KIND == 2 || KIND == 3) dif_stages<R>(v, bases);
     if (KIND == 3) {
       // s = 1: the group's elements are contiguous in the spectrum's storage order
 #pragma unroll
       for (int k = 0; k < E; ++k) v[k] = cmul(v[k], hq[i0 + k]);
     }
-    if (KIND == 1 || KIND == 3 || KIND == 4) dit_stages<R>(v, tw, logc, logs, j0);
+    if (KIND == 1 || KIND == 3 || KIND == 4) dit_stages<R>(v, bases);
     if (KIND == 2) {
 #pragma unroll
       for (int k = 0; k < E; ++k) out[i0 + k * s] = v[k];
@@ -173,11 +184,11 @@ __device__ __forceinline__ void fft_pass(float2* a, const float2* tw, int logc, 
 }
 
 template <int KIND>
-__device__ __forceinline__ void run_pass(int r, float2* a, const float2* tw, int logc, int logs, float2* out,
+__device__ __forceinline__ void run_pass(int r, float2* a, const float2* tp, int logc, int logs, float2* out,
                                          const float2* hq, const float2* lo, const float2* hi, int logc1) {
-  if (r == 1) fft_pass<1, KIND>(a, tw, logc, logs, out, hq, lo, hi, logc1);
-  else if (r == 2) fft_pass<2, KIND>(a, tw, logc, logs, out, hq, lo, hi, logc1);
-  else fft_pass<3, KIND>(a, tw, logc, logs, out, hq, lo, hi, logc1);
+  if (r == 1) fft_pass<1, KIND>(a, tp, logc, logs, out, hq, lo, hi, logc1);
+  else if (r == 2) fft_pass<2, KIND>(a, tp, logc, logs, out, hq, lo, hi, logc1);
+  else fft_pass<3, KIND>(a, tp, logc, logs, out, hq, lo, hi, logc1);
 }
 
 // Split log2(c) stages into passes of at most 3 (as even as possible); forward: largest spans
@@ -202,14 +213,26 @@ __global__ void __launch_bounds__(kFftThreads, 2) fftconv_slice_kernel(const Fft
   const int c = p.c;
   const int logc1 = p.logc < 6 ? p.logc : 6;          // n = n_lo + C1 n_hi, C1 = min(c, 64)
   const int c1 = 1 << logc1;
+  int radix[5], toff[6];
+  const int np = fft_passes(p.logc, radix);
   float2* a = fsm;                           // c values at pidx(i)
-  float2* tw = fsm + c + c / 16;             // c / 2 twiddles w_c^m
-  float2* cf = tw + c / 2;                   // N cross-rank coefficients w_2N^(r q)
+  float2* tpass = fsm + c + c / 16;          // per pass p: w_(s_p 2^R_p)^j0, j0 < s_p (<= c / 4 + 1 in all)
+  {
+    int logs = p.logc, off = 0;
+    for (int i = 0; i < np; ++i) {
+      logs -= radix[i];
+      toff[i] = off;
+      // w_(s 2^R)^j0 = w_c^(j0 c / (s 2^R)); s = 2^logs
+      for (int j0 = threadIdx.x; j0 < (1 << logs); j0 += kFftThreads)
+        tpass[off + j0] = p.twc[j0 << (p.logc - logs - radix[i])];
+      off += 1 << logs;
+    }
+    toff[np] = off;
+  }
+  float2* cf = tpass + c / 4 + 16;           // N cross-rank coefficients w_2N^(r q)
   float2* lo = cf + kFftMaxN;                // w_2L^(u q), u < C1
   float2* hi = lo + 64;                      // w_2L^(C1 v q), v < c / C1 (<= 128)
 
-#pragma unroll 8
-  for (int m = threadIdx.x; m < c / 2; m += kFftThreads) tw[m] = p.twc[m];
   // w_2N^(r q) = w_2L^((r q mod 2N) c); lo/hi: every index below 2L (u q < C1 2N <= 2L, C1 v q < c 2N)
   for (int r = threadIdx.x; r < p.N; r += kFftThreads) cf[r] = p.tw2l[((r * q) % Q) * c];
   if (threadIdx.x < c1) lo[threadIdx.x] = p.tw2l[threadIdx.x * q];
@@ -265,32 +288,30 @@ __global__ void __launch_bounds__(kFftThreads, 2) fftconv_slice_kernel(const Fft
   }
   __syncthreads();
 
-  int radix[5];
-  const int np = fft_passes(p.logc, radix);
   const long long slice = (static_cast<long long>(row) * Q + q) * c;
   int logs = p.logc;
   for (int i = 0; i + 1 < np; ++i) {
     logs -= radix[i];
-    run_pass<0>(radix[i], a, tw, p.logc, logs, nullptr, nullptr, nullptr, nullptr, 0);
+    run_pass<0>(radix[i], a, tpass + toff[i], p.logc, logs, nullptr, nullptr, nullptr, nullptr, 0);
     __syncthreads();
   }
   // logs is now radix[np-1]: the last pass has s = 1
   if (MODE == 0) {
-    run_pass<2>(radix[np - 1], a, tw, p.logc, 0, p.spec + slice, nullptr, nullptr, nullptr, 0);
+    run_pass<2>(radix[np - 1], a, tpass + toff[np - 1], p.logc, 0, p.spec + slice, nullptr, nullptr, nullptr, 0);
     return;
   }
   const float2* hq = p.spec + (static_cast<long long>(ch) * Q + q) * c;
-  run_pass<3>(radix[np - 1], a, tw, p.logc, 0, nullptr, hq, nullptr, nullptr, 0);
+  run_pass<3>(radix[np - 1], a, tpass + toff[np - 1], p.logc, 0, nullptr, hq, nullptr, nullptr, 0);
   __syncthreads();
   logs = radix[np - 1];
   for (int i = np - 2; i >= 1; --i) {
-    run_pass<1>(radix[i], a, tw, p.logc, logs, nullptr, nullptr, nullptr, nullptr, 0);
+    run_pass<1>(radix[i], a, tpass + toff[i], p.logc, logs, nullptr, nullptr, nullptr, nullptr, 0);
     logs += radix[i];
     __syncthreads();
   }
   if (np >= 2) {
     // the last inverse pass writes w_q(n) = w_2L^(-n q) * (local inverse) straight to global
-    run_pass<4>(radix[0], a, tw, p.logc, logs, p.w + slice, nullptr, lo, hi, logc1);
+    run_pass<4>(radix[0], a, tpass + toff[0], p.logc, logs, p.w + slice, nullptr, lo, hi, logc1);
   } else {
     for (int n = threadIdx.x; n < c; n += kFftThreads)
       p.w[slice + n] = cmul_conj(a[pidx(n)], cmul(lo[n & (c1 - 1)], hi[n >> logc1]));
@@ -338,7 +359,7 @@ __global__ void __launch_bounds__(kFftThreads) fftconv_inverse_kernel(const FftI
 }
 
 __host__ __device__ constexpr size_t fftconv_smem_bytes(int c, int N) {
-  return (static_cast<size_t>(c) + c / 16 + c / 2 + kFftMaxN + 64 + 128) * sizeof(float2);
+  return (static_cast<size_t>(c) + c / 16 + c / 4 + 16 + kFftMaxN + 64 + 128) * sizeof(float2);
 }
 
 }  // namespace cpattn
