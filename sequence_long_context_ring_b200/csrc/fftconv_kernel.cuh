@@ -82,9 +82,12 @@ __device__ __forceinline__ float2 rot(float2 z) {
   }
 }
 
-// Shared-memory index of element i: one float2 of padding per 16 keeps the power-of-two
-// strides of the passes off a single bank.
-__device__ __forceinline__ int pidx(int i) { return i + (i >> 4); }
+// Shared-memory index of element i: within each row of 16 float2 (128 bytes, one pass over
+// the banks) the position is XORed with 5 x the row number.  A bijection inside every row, so
+// no padding; chosen by enumerating the half-warp access patterns of every pass (radix 8 at
+// spans 1024/128/16 or 256/32/4, radix 4 at spans 4/1, the cross stage's 8-sample runs, the
+// contiguous reads): each lands on 16 distinct bank pairs.
+__device__ __forceinline__ int pidx(int i) { return i ^ (((i >> 4) * 5) & 15); }
 
 // The twiddle of stage t (span s 2^t) for group element k: w_2hs^(j0 + s m) = base * w_(2^(t+1))^m,
 // m = k mod 2^t, base = w_2hs^j0 (one table read per stage).
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(kFftThreads, 2) fftconv_slice_kernel(const Fft
   int radix[5], toff[6];
   const int np = fft_passes(p.logc, radix);
   float2* a = fsm;                           // c values at pidx(i)
-  float2* tpass = fsm + c + c / 16;          // per pass p: w_(s_p 2^R_p)^j0, j0 < s_p (<= c / 4 + 1 in all)
+  float2* tpass = fsm + c;                   // per pass p: w_(s_p 2^R_p)^j0, j0 < s_p (<= c / 4 + 1 in all)
   {
     int logs = p.logc, off = 0;
     for (int i = 0; i < np; ++i) {
@@ -359,7 +362,7 @@ __global__ void __launch_bounds__(kFftThreads) fftconv_inverse_kernel(const FftI
 }
 
 __host__ __device__ constexpr size_t fftconv_smem_bytes(int c, int N) {
-  return (static_cast<size_t>(c) + c / 16 + c / 4 + 16 + kFftMaxN + 64 + 128) * sizeof(float2);
+  return (static_cast<size_t>(c) + c / 4 + 16 + kFftMaxN + 64 + 128) * sizeof(float2);
 }
 
 }  // namespace cpattn
