@@ -60,7 +60,8 @@ struct DqItem {
   int b, h, g, r, row0, q_end, n_diag, n_tiles;
 };
 
-// Work items longest first: last chunk, last query tiles (the causal work grows with the row).
+// Work items (batch, KV head)-major, then longest first: last chunk, last query tiles (the
+// causal work grows with the row).
 __device__ __forceinline__ DqItem decode_dq_item(const DqParams& p) {
   DqItem it;
   // (batch, KV head)-major: the CTAs in flight are the query tiles of one KV group's heads and
