@@ -5,7 +5,6 @@ import numpy as np
 import pytest
 import torch
 
-from sequence_long_context_ring_b200 import synth
 from sequence_long_context_ring_b200.binding import Plan, CpError
 
 from _helpers import to_dev, inputs
