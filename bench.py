@@ -10,8 +10,9 @@ needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload c3]
 
-Multi-GPU: the benchmark spec keeps every virtual rank of the problem on one GPU, so N > 1 runs
-N independent replicas (one per GPU, weak scaling); value = total FLOPs / max-over-ranks time.
+Multi-GPU: every virtual rank of a problem runs on one GPU (the path has no exchange between
+GPUs), so N > 1 runs N independent replicas (one per GPU, weak scaling); value = total FLOPs /
+max-over-ranks time.
 --impl reference times the fp64 CPU oracle on a bounded row sample of the same workload.
 """
 from __future__ import annotations
