@@ -179,3 +179,47 @@ def test_fftconv_workspace_and_cost():
     assert flops > 0
     lib = binding.lib()
     assert lib.cp_fftconv_fwd(p._h, None, None, None, None, 0, None) == binding.CP_ERR_INVALID_ARG
+
+
+# ---- the host-buffer forward (cp_attn_fwd_host): argument checks run before any CUDA call ----
+def _host_desc(shape, dtype_code, strides=None):
+    d = binding.CpTensor()
+    d.data = 4096            # never dereferenced: the checks reject the call first
+    d.dtype = dtype_code
+    d.ndim = len(shape)
+    st = strides
+    if st is None:
+        st, acc = [], 1
+        for n in reversed(shape):
+            st.insert(0, acc)
+            acc *= n
+    for i, n in enumerate(shape):
+        d.shape[i] = n
+        d.stride[i] = st[i]
+    return d
+
+
+def test_host_forward_workspace_size_and_argument_checks():
+    B, Hq, Hkv, L, d = 1, 8, 2, 512, 64
+    plan = Plan(B, Hq, Hkv, L, d, n_cp=4)
+    a256 = lambda n: (n + 255) // 256 * 256
+    nq, nkv = B * Hq * L * d, B * Hkv * L * d
+    assert plan.host_workspace_size() == 2 * a256(nq * 2) + 2 * a256(nkv * 2) + a256(B * Hq * L * 4)
+    lib = binding.lib()
+    q = _host_desc((B, Hq, L, d), binding.CP_BF16)
+    k = _host_desc((B, Hkv, L, d), binding.CP_BF16)
+    o = _host_desc((B, Hq, L, d), binding.CP_BF16)
+    lse = _host_desc((B, Hq, L), binding.CP_FP32)
+    r = ctypes.byref
+    # workspace missing
+    assert lib.cp_attn_fwd_host(plan._h, r(q), r(k), r(k), r(o), r(lse), None, 0, None) == binding.CP_ERR_WORKSPACE
+    # wrong shape, wrong dtype, non-canonical strides
+    bad = _host_desc((B, Hq, L, d + 8), binding.CP_BF16)
+    assert lib.cp_attn_fwd_host(plan._h, r(bad), r(k), r(k), r(o), r(lse), None, 0, None) == binding.CP_ERR_INVALID_ARG
+    badt = _host_desc((B, Hq, L), binding.CP_BF16)
+    assert lib.cp_attn_fwd_host(plan._h, r(q), r(k), r(k), r(o), r(badt), None, 0, None) == binding.CP_ERR_INVALID_ARG
+    strided = _host_desc((B, Hq, L, d), binding.CP_BF16, [Hq * L * d * 2, L * d * 2, d * 2, 1])
+    assert lib.cp_attn_fwd_host(plan._h, r(strided), r(k), r(k), r(o), r(lse), None, 0, None) == binding.CP_ERR_ALIGNMENT
+    # ring plans only
+    uly = Plan(B, Hq, Hkv, L, d, n_cp=2, mode="ulysses")
+    assert lib.cp_attn_fwd_host(uly._h, r(q), r(k), r(k), r(o), r(lse), None, 0, None) == binding.CP_ERR_UNSUPPORTED
