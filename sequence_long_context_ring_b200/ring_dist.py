@@ -1,0 +1,86 @@
+"""Ring attention across GPUs, one rank per GPU ("05. 長系列の分散学習（Context Parallelism）",
+"ring attention: key/value をリングで回す", steps 1-4: each rank keeps its queries, passes its
+key/value shard to the next rank, computes a partial attention against the shard it holds at
+each step, and merges the partials with the online-softmax statistics).
+
+Rank r holds the query shard Q_r and the key/value shard (K_r, V_r) of a sequence split into
+N = world contiguous shards.  At step s = 0 .. N-1 it holds the shard of rank j = (r - s) mod N:
+while the partial of Q_r against it runs on the GPU (the library's ring-step kernel with a
+one-chunk plan: causal at j = r, full for j < r, skipped for j > r under the causal mask), the
+shard is sent on to rank r + 1 and the next one received from rank r - 1 into a second buffer
+(one message of [2, B, Hkv, c, d] per step, point-to-point over the process group: NCCL over
+NVLink on GPUs).  The partials merge into an fp32 accumulator with the library's LSE merge.
+
+The exchange lands every remote shard in this rank's own memory before a kernel reads it;
+no kernel reads a peer's memory.
+"""
+from __future__ import annotations
+
+from typing import Callable, Optional
+
+import torch
+import torch.distributed as dist
+
+from .binding import Plan, lse_merge
+
+
+class _PlanCache:
+    """One-chunk plans by (shape, diagonal, scale): plans are host objects, cheap to keep."""
+
+    def __init__(self):
+        self._plans = {}
+
+    def get(self, B, Hq, Hkv, c, d, diagonal, scale):
+        key = (B, Hq, Hkv, c, d, bool(diagonal), float(scale))
+        p = self._plans.get(key)
+        if p is None:
+            p = Plan(B, Hq, Hkv, c, d, n_cp=1, causal=bool(diagonal), scale=float(scale))
+            self._plans[key] = p
+        return p
+
+
+_plans = _PlanCache()
+
+
+def cuda_partial(q, k, v, diagonal: bool, scale: float):
+    """The partial (fp32 O normalised, LSE) of q [B, Hq, c, d] against one key/value shard
+    k, v [B, Hkv, c, d]: the ring-step kernel on a one-chunk plan (causal mask at the
+    diagonal shard, none below it)."""
+    B, Hq, c, d = q.shape
+    return _plans.get(B, Hq, k.shape[1], c, d, diagonal, scale).ring_step(0, 0, q, k, v)
+
+
+def ring_attention(q, k, v, group=None, *, causal: bool = True, scale: float = 0.0,
+                   partial_fn: Optional[Callable] = None, merge_fn: Optional[Callable] = None):
+    """This rank's share of ring attention over the process group.
+
+    q [B, Hq, c, d], k, v [B, Hkv, c, d]: this rank's shards (rank r holds sequence positions
+    [r c, (r+1) c)).  Returns (O fp32 [B, Hq, c, d] normalised, LSE fp32 [B, Hq, c]) of this
+    rank's queries over the whole sequence.  partial_fn(q, k, v, diagonal, scale) -> (O, LSE) and
+    merge_fn(acc_o, acc_lse, o, lse) (in place) default to the library's kernels."""
+    partial_fn = partial_fn or cuda_partial
+    merge_fn = merge_fn or lse_merge
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    nxt, prv = (rank + 1) % world, (rank - 1) % world
+    if group is not None:
+        nxt, prv = dist.get_global_rank(group, nxt), dist.get_global_rank(group, prv)
+    kv_cur = torch.stack([k, v]).contiguous()       # one message: [2, B, Hkv, c, d]
+    kv_nxt = torch.empty_like(kv_cur)
+    B, Hq, c, d = q.shape
+    acc_o = torch.zeros((B, Hq, c, d), dtype=torch.float32 if q.is_cuda else torch.float64, device=q.device)
+    acc_l = torch.full((B, Hq, c), -float("inf"), dtype=acc_o.dtype, device=q.device)
+    for s in range(world):
+        j = (rank - s) % world
+        reqs = []
+        if s < world - 1:
+            # pass the shard held now to the next rank, receive the next one from the previous
+            reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, kv_cur, nxt, group),
+                                           dist.P2POp(dist.irecv, kv_nxt, prv, group)])
+        if not (causal and j > rank):
+            po, pl = partial_fn(q, kv_cur[0], kv_cur[1], causal and j == rank, scale)
+            merge_fn(acc_o, acc_l, po, pl)
+        for r in reqs:
+            r.wait()
+        kv_cur, kv_nxt = kv_nxt, kv_cur
+    return acc_o, acc_l
