@@ -33,7 +33,7 @@ def _rank(rank, world, port, out):
 
 def test_max_over_ranks_and_whole_job_value_gloo():
     port = 29500 + os.getpid() % 2000
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         out = man.dict()
         mp.spawn(_rank, args=(2, port, out), nprocs=2, join=True)
         res = dict(out)

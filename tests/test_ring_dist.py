@@ -70,7 +70,7 @@ def _rank(rank, world, port, causal, out):
 def test_ring_across_processes_equals_full_attention(world, causal):
     import oracle
     port = 29600 + (os.getpid() * 7 + world * 13 + int(causal)) % 2000
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         out = man.dict()
         mp.spawn(_rank, args=(world, port, causal, out), nprocs=world, join=True)
         res = dict(out)
