@@ -11,6 +11,13 @@ shard is sent on to rank r + 1 and the next one received from rank r - 1 into a 
 (one message of [2, B, Hkv, c, d] per step, point-to-point over the process group: NCCL over
 NVLink on GPUs).  The partials merge into an fp32 accumulator with the library's LSE merge.
 
+Two-shard splits (§5 因果モデルの負荷分散): with split = "zigzag" (rank r holds shards r and
+2N-1-r of 2N) or "striped" (shards r and r+N), every rank's local rows are its two shards in
+that order, each w = c/2 rows, and so are the key/value rows it passes on.  The partial of a
+step is then the merge of up to four shard-pair partials: shard a's queries against shard b's
+keys are full when b < a, masked (key <= query) when b == a, and skipped when b > a.  Every
+step carries the same causal work under zig-zag, which is why the split is used.
+
 The exchange lands every remote shard in this rank's own memory before a kernel reads it;
 no kernel reads a peer's memory.
 """
@@ -50,13 +57,23 @@ def cuda_partial(q, k, v, diagonal: bool, scale: float):
     return _plans.get(B, Hq, k.shape[1], c, d, diagonal, scale).ring_step(0, 0, q, k, v)
 
 
-def ring_attention(q, k, v, group=None, *, causal: bool = True, scale: float = 0.0,
+def shards_of_rank(split: str, n: int, r: int):
+    """The two shard indices (of 2n) held by rank r under a two-shard split."""
+    if split == "zigzag":
+        return (r, 2 * n - 1 - r)
+    if split == "striped":
+        return (r, r + n)
+    raise ValueError(f"unknown split {split!r}")
+
+
+def ring_attention(q, k, v, group=None, *, causal: bool = True, scale: float = 0.0, split: str = "contiguous",
                    partial_fn: Optional[Callable] = None, merge_fn: Optional[Callable] = None):
     """This rank's share of ring attention over the process group.
 
-    q [B, Hq, c, d], k, v [B, Hkv, c, d]: this rank's shards (rank r holds sequence positions
-    [r c, (r+1) c)).  Returns (O fp32 [B, Hq, c, d] normalised, LSE fp32 [B, Hq, c]) of this
-    rank's queries over the whole sequence.  partial_fn(q, k, v, diagonal, scale) -> (O, LSE) and
+    q [B, Hq, c, d], k, v [B, Hkv, c, d]: this rank's rows (contiguous: sequence positions
+    [r c, (r+1) c); zigzag / striped: its two shards of c/2 positions, in order).  Returns
+    (O [B, Hq, c, d] normalised, LSE [B, Hq, c]) of this rank's queries over the whole
+    sequence, in fp32 on the GPU.  partial_fn(q, k, v, diagonal, scale) -> (O, LSE) and
     merge_fn(acc_o, acc_lse, o, lse) (in place) default to the library's kernels."""
     partial_fn = partial_fn or cuda_partial
     merge_fn = merge_fn or lse_merge
@@ -68,6 +85,8 @@ def ring_attention(q, k, v, group=None, *, causal: bool = True, scale: float = 0
     kv_cur = torch.stack([k, v]).contiguous()       # one message: [2, B, Hkv, c, d]
     kv_nxt = torch.empty_like(kv_cur)
     B, Hq, c, d = q.shape
+    if split != "contiguous" and c % 2:
+        raise ValueError("a two-shard split needs an even number of local rows")
     acc_o = torch.zeros((B, Hq, c, d), dtype=torch.float32 if q.is_cuda else torch.float64, device=q.device)
     acc_l = torch.full((B, Hq, c), -float("inf"), dtype=acc_o.dtype, device=q.device)
     for s in range(world):
@@ -77,9 +96,20 @@ def ring_attention(q, k, v, group=None, *, causal: bool = True, scale: float = 0
             # pass the shard held now to the next rank, receive the next one from the previous
             reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, kv_cur, nxt, group),
                                            dist.P2POp(dist.irecv, kv_nxt, prv, group)])
-        if not (causal and j > rank):
-            po, pl = partial_fn(q, kv_cur[0], kv_cur[1], causal and j == rank, scale)
-            merge_fn(acc_o, acc_l, po, pl)
+        if split == "contiguous":
+            if not (causal and j > rank):
+                po, pl = partial_fn(q, kv_cur[0], kv_cur[1], causal and j == rank, scale)
+                merge_fn(acc_o, acc_l, po, pl)
+        else:
+            w = c // 2
+            for qa, a in enumerate(shards_of_rank(split, world, rank)):
+                for kb, b in enumerate(shards_of_rank(split, world, j)):
+                    if causal and b > a:
+                        continue
+                    qs, ks = slice(qa * w, (qa + 1) * w), slice(kb * w, (kb + 1) * w)
+                    po, pl = partial_fn(q[:, :, qs], kv_cur[0][:, :, ks], kv_cur[1][:, :, ks],
+                                        causal and b == a, scale)
+                    merge_fn(acc_o[:, :, qs], acc_l[:, :, qs], po, pl)
         for r in reqs:
             r.wait()
         kv_cur, kv_nxt = kv_nxt, kv_cur

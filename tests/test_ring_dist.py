@@ -1,8 +1,9 @@
 """The ring across processes ("05. 長系列の分散学習（Context Parallelism）", ring attention steps
-1-4) on CPU: gloo ranks, one per shard, run ring_dist.ring_attention's exchange schedule
-(send the held key/value shard to the next rank, receive the next from the previous, N - 1
-exchanges, causal skip above the diagonal) with the oracle's chunk partial and merge standing
-in for the GPU kernels.  Every rank's result must equal full attention on its rows.
+1-4, and the two-shard splits of §5) on CPU: gloo ranks, one per shard, run
+ring_dist.ring_attention's exchange schedule (send the held key/value rows to the next rank,
+receive the next from the previous, N - 1 exchanges, causal skip above the diagonal, shard
+pairs under zig-zag / striped) with the oracle's chunk partial and merge standing in for the
+GPU kernels.  Every rank's result must equal full attention on its rows.
 
 On GPUs the same schedule runs the library's ring-step and merge kernels over NCCL; that form
 needs several GPUs in one job and is not run here."""
@@ -17,13 +18,22 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _inputs(world, B=1, Hq=4, Hkv=2, c=6, d=8):
+    # c = 6 local rows: shards of 3 under a two-shard split
     rng = np.random.default_rng(100 + world)
     L = c * world
     return (rng.standard_normal((B, Hq, L, d)), rng.standard_normal((B, Hkv, L, d)),
             rng.standard_normal((B, Hkv, L, d)))
 
 
-def _rank(rank, world, port, causal, out):
+def _positions(split, world, L, r):
+    from oracle import split as osp
+    if split == "contiguous":
+        c = L // world
+        return np.arange(r * c, (r + 1) * c)
+    return osp.rank_positions(split, world, L, r)
+
+
+def _rank(rank, world, port, causal, split, out):
     import torch
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
@@ -36,9 +46,8 @@ def _rank(rank, world, port, causal, out):
         q, k, v = _inputs(world)
         B, Hq, L, d = q.shape
         G = Hq // k.shape[1]
-        c = L // world
-        sl = slice(rank * c, (rank + 1) * c)
-        qr, kr, vr = (torch.from_numpy(np.ascontiguousarray(x[:, :, sl])) for x in (q, k, v))
+        pos = _positions(split, world, L, rank)
+        qr, kr, vr = (torch.from_numpy(np.ascontiguousarray(x[:, :, pos])) for x in (q, k, v))
         calls = []
 
         def partial(qq, kk, vv, diagonal, scale):
@@ -59,31 +68,47 @@ def _rank(rank, world, port, causal, out):
             acc_o.copy_(torch.from_numpy(o2))
             acc_l.copy_(torch.from_numpy(l2))
 
-        o, lse = ring_dist.ring_attention(qr, kr, vr, causal=causal, partial_fn=partial, merge_fn=merge)
+        o, lse = ring_dist.ring_attention(qr, kr, vr, causal=causal, split=split, partial_fn=partial, merge_fn=merge)
         out[rank] = (o.numpy(), lse.numpy(), calls)
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [1, 2, 3, 4])
-@pytest.mark.parametrize("causal", [True, False])
-def test_ring_across_processes_equals_full_attention(world, causal):
+@pytest.mark.parametrize("world,causal,split", [
+    (1, True, "contiguous"), (2, True, "contiguous"), (3, True, "contiguous"), (4, True, "contiguous"),
+    (1, False, "contiguous"), (3, False, "contiguous"),
+    (2, True, "zigzag"), (3, True, "zigzag"), (4, True, "zigzag"), (3, True, "striped"), (2, False, "zigzag"),
+])
+def test_ring_across_processes_equals_full_attention(world, causal, split):
     import oracle
-    port = 29600 + (os.getpid() * 7 + world * 13 + int(causal)) % 2000
+    port = 29600 + (os.getpid() * 7 + world * 13 + int(causal) + 3 * len(split)) % 2000
     with mp.get_context("spawn").Manager() as man:
         out = man.dict()
-        mp.spawn(_rank, args=(world, port, causal, out), nprocs=world, join=True)
+        mp.spawn(_rank, args=(world, port, causal, split, out), nprocs=world, join=True)
         res = dict(out)
     q, k, v = _inputs(world)
+    L = q.shape[2]
     o_ref, l_ref = oracle.attention_full(q, k, v, causal=causal)
-    c = q.shape[2] // world
     for r in range(world):
         o, lse, calls = res[r]
-        np.testing.assert_allclose(o, o_ref[:, :, r * c:(r + 1) * c], atol=1e-12)
-        np.testing.assert_allclose(lse, l_ref[:, :, r * c:(r + 1) * c], atol=1e-12)
-        # causal: rank r computes its r + 1 shards at or below the diagonal (the diagonal one
-        # masked, first) and skips the rest; otherwise all N shards, none masked
-        if causal:
-            assert calls == [True] + [False] * r
-        else:
-            assert calls == [False] * world
+        pos = _positions(split, world, L, r)
+        np.testing.assert_allclose(o, o_ref[:, :, pos], atol=1e-12)
+        np.testing.assert_allclose(lse, l_ref[:, :, pos], atol=1e-12)
+        if split == "contiguous":
+            # causal: rank r computes its r + 1 shards at or below the diagonal (the diagonal
+            # one masked, first) and skips the rest; otherwise all N shards, none masked
+            assert calls == ([True] + [False] * r if causal else [False] * world)
+        elif causal:
+            # two shards per rank: the shard pairs at or below the diagonal, one masked pair per
+            # own shard; under zig-zag every step but the first carries 2 full pairs
+            n_pairs = sum(1 for s in range(world)
+                          for a in ring_dist_shards(split, world, r)
+                          for b in ring_dist_shards(split, world, (r - s) % world) if b <= a)
+            assert len(calls) == n_pairs and sum(calls) == 2
+            if split == "zigzag":
+                assert n_pairs == 3 + 2 * (world - 1)
+
+
+def ring_dist_shards(split, world, r):
+    from oracle import split as osp
+    return osp.shards_of_rank(split, world, r)
