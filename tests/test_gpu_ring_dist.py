@@ -32,5 +32,10 @@ def test_one_rank_ring_matches_the_oracle(cuda_lib):
         torch.cuda.synchronize()
         o2_ref, l2_ref = oracle.attention_full(*(to_f64(to_dev(x)) for x in (q, k, v)), causal=False)
         assert_attn_close(to_f64(o2), o2_ref, to_f64(l2), l2_ref, "one-rank ring, non-causal")
+        # zig-zag with one rank: its two shards (first and second half) as shard pairs on
+        # strided views -- (0,0) masked, (1,0) full, (1,1) masked -- equal full causal attention
+        o3, l3 = ring_dist.ring_attention(to_dev(q), to_dev(k), to_dev(v), split="zigzag")
+        torch.cuda.synchronize()
+        assert_attn_close(to_f64(o3), o_ref, to_f64(l3), l_ref, "one-rank zig-zag ring")
     finally:
         dist.destroy_process_group()
