@@ -112,3 +112,62 @@ def test_ring_across_processes_equals_full_attention(world, causal, split):
 def ring_dist_shards(split, world, r):
     from oracle import split as osp
     return osp.shards_of_rank(split, world, r)
+
+
+def _rank_groups(rank, world, port, out):
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from sequence_long_context_ring_b200 import ring_dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # two independent rings of two ranks each: global ranks {0, 2} and {1, 3}, so the
+        # neighbours inside a group are not the neighbours in the world
+        groups = [dist.new_group([0, 2]), dist.new_group([1, 3])]
+        g = rank % 2
+        gr = rank // 2
+        q, k, v = _inputs(10 + g)                 # each group attends over its own problem
+        B, Hq, L, d = q.shape
+        G = Hq // k.shape[1]
+        c = L // 2
+        sl = slice(gr * c, (gr + 1) * c)
+        qr, kr, vr = (torch.from_numpy(np.ascontiguousarray(x[:, :, sl])) for x in (q, k, v))
+
+        def partial(qq, kk, vv, diagonal, scale):
+            qq, kk, vv = qq.numpy(), kk.numpy(), vv.numpy()
+            o = np.zeros(qq.shape)
+            lse = np.zeros(qq.shape[:3])
+            for b in range(B):
+                for h in range(Hq):
+                    o[b, h], lse[b, h] = oracle.chunk_partial(qq[b, h], kk[b, h // G], vv[b, h // G], 0, 0,
+                                                              causal=bool(diagonal))
+            return torch.from_numpy(o), torch.from_numpy(lse)
+
+        def merge(acc_o, acc_l, po, pl):
+            o2, l2 = oracle.lse_merge(acc_o.numpy(), acc_l.numpy(), po.numpy(), pl.numpy())
+            acc_o.copy_(torch.from_numpy(o2))
+            acc_l.copy_(torch.from_numpy(l2))
+
+        o, lse = ring_dist.ring_attention(qr, kr, vr, groups[g], partial_fn=partial, merge_fn=merge)
+        out[rank] = (o.numpy(), lse.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rings_in_process_subgroups():
+    import oracle
+    port = 29650 + (os.getpid() * 11) % 2000
+    with mp.get_context("spawn").Manager() as man:
+        out = man.dict()
+        mp.spawn(_rank_groups, args=(4, port, out), nprocs=4, join=True)
+        res = dict(out)
+    for rank in range(4):
+        g, gr = rank % 2, rank // 2
+        q, k, v = _inputs(10 + g)
+        o_ref, l_ref = oracle.attention_full(q, k, v)
+        c = q.shape[2] // 2
+        np.testing.assert_allclose(res[rank][0], o_ref[:, :, gr * c:(gr + 1) * c], atol=1e-12)
+        np.testing.assert_allclose(res[rank][1], l_ref[:, :, gr * c:(gr + 1) * c], atol=1e-12)
