@@ -142,6 +142,20 @@ def _stream(stream) -> Optional[int]:
     return getattr(stream, "cuda_stream", stream)
 
 
+def _on_device(*tensors) -> None:
+    """The device entry points dereference their pointers in kernels: a host tensor there would
+    be a GPU memory fault, so it is refused before the call."""
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise ValueError("expected a CUDA tensor (this call's kernels read and write device memory)")
+
+
+def _on_host(*tensors) -> None:
+    for t in tensors:
+        if t is not None and t.is_cuda:
+            raise ValueError("expected a host tensor (this call copies host memory in and out itself)")
+
+
 class Plan:
     """A cp_attn plan: validated problem geometry (host only until the first launch)."""
 
@@ -191,6 +205,7 @@ class Plan:
 
     def fwd(self, q, k, v, o=None, lse=None, ws=None, stream=None):
         """Forward; returns (o, lse).  Layouts per mode (see cp_attn.h)."""
+        _on_device(q, k, v, o, lse, ws)
         c = self.cfg
         if o is None:
             o = torch.empty_like(q)
@@ -214,6 +229,8 @@ class Plan:
         """Forward of a ring plan on HOST tensors (contiguous, preferably pinned): the library
         copies in, computes and copies out, overlapping the transfers with the kernels.  ws:
         device staging of host_workspace_size() bytes."""
+        _on_host(q, k, v, o, lse)
+        _on_device(ws)
         if ws is None:
             ws = torch.empty(self.host_workspace_size(), dtype=torch.uint8, device="cuda")
         td = [tensor_desc(t) for t in (q, k, v, o, lse)]
@@ -225,6 +242,7 @@ class Plan:
         """Forward of a Ulysses / 2D plan through cp_attn_fwd_noalloc: the library uses its
         static 64 MiB scratch instead of a workspace and allocates nothing.  o and lse must
         be given (preallocated by the caller)."""
+        _on_device(q, k, v, o, lse)
         td = [tensor_desc(t) for t in (q, k, v, o, lse)]
         _check(lib().cp_attn_fwd_noalloc(self._h, *[ctypes.byref(t) for t in td], _stream(stream)),
                "cp_attn_fwd_noalloc")
@@ -232,6 +250,7 @@ class Plan:
 
     def bwd(self, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, ws=None, stream=None):
         """Backward; returns (dq, dk, dv)."""
+        _on_device(q, k, v, o, lse, dout, dq, dk, dv, ws)
         dq = torch.empty_like(q) if dq is None else dq
         dk = torch.empty_like(k) if dk is None else dk
         dv = torch.empty_like(v) if dv is None else dv
@@ -246,6 +265,7 @@ class Plan:
 
     def ring_step(self, rank: int, step: int, q, k, v, o_part=None, lse_part=None, stream=None):
         """One ring step's fp32 partial (O normalised, LSE) of query chunk `rank`."""
+        _on_device(q, k, v, o_part, lse_part)
         c = self.cfg
         ch = c.L // c.n_cp
         if o_part is None:
@@ -265,6 +285,7 @@ class Plan:
 
 
 def lse_merge(o_acc, lse_acc, o_part, lse_part, stream=None) -> None:
+    _on_device(o_acc, lse_acc, o_part, lse_part)
     td = [tensor_desc(t) for t in (o_acc, lse_acc, o_part, lse_part)]
     _check(lib().cp_lse_merge(*[ctypes.byref(t) for t in td], _stream(stream)), "cp_lse_merge")
 
@@ -272,6 +293,7 @@ def lse_merge(o_acc, lse_acc, o_part, lse_part, stream=None) -> None:
 def seq2head(n_ranks: int, x, out=None, stream=None, split: str = "contiguous"):
     """[B, L, H, d] (rank-major under a two-shard split) -> [B, H, L, d] in position order
     (Ulysses all-to-all, bit-exact)."""
+    _on_device(x, out)
     if out is None:
         B, L, H, d = x.shape
         out = torch.empty((B, H, L, d), dtype=x.dtype, device=x.device)
@@ -287,6 +309,7 @@ def seq2head(n_ranks: int, x, out=None, stream=None, split: str = "contiguous"):
 def head2seq(n_ranks: int, x, out=None, stream=None, split: str = "contiguous"):
     """[B, H, L, d] in position order -> [B, L, H, d] (rank-major under a two-shard split),
     the inverse all-to-all, bit-exact."""
+    _on_device(x, out)
     if out is None:
         B, H, L, d = x.shape
         out = torch.empty((B, L, H, d), dtype=x.dtype, device=x.device)
@@ -323,6 +346,7 @@ class ConvPlan:
 
     def fwd(self, x, h, y=None, stream=None):
         """y = x * h over the whole sequence [B, D, L] (every virtual rank, halos in place)."""
+        _on_device(x, h, y)
         y = torch.empty_like(x) if y is None else y
         td = [tensor_desc(t) for t in (x, h, y)]
         _check(lib().cp_conv_fir_fwd(self._h, *[ctypes.byref(t) for t in td], _stream(stream)), "cp_conv_fir_fwd")
@@ -330,6 +354,7 @@ class ConvPlan:
 
     def shard(self, rank: int, x, halo, h, y=None, stream=None):
         """One rank's shard [B, D, L/n_cp] with the halo [B, D, lh-1] from rank-1 (None at rank 0)."""
+        _on_device(x, halo, h, y)
         y = torch.empty_like(x) if y is None else y
         dx, dh, dy = tensor_desc(x), tensor_desc(h), tensor_desc(y)
         dg = ctypes.byref(tensor_desc(halo)) if halo is not None else None
@@ -375,6 +400,7 @@ class FftConvPlan:
 
     def fwd(self, x, h, y=None, ws=None, stream=None):
         """y = x * h, x [B, D, L], h [D, L] (bf16)."""
+        _on_device(x, h, y, ws)
         y = torch.empty_like(x) if y is None else y
         ws = self.workspace(x.device) if ws is None else ws
         td = [tensor_desc(t) for t in (x, h, y)]

@@ -223,3 +223,23 @@ def test_host_forward_workspace_size_and_argument_checks():
     # ring plans only
     uly = Plan(B, Hq, Hkv, L, d, n_cp=2, mode="ulysses")
     assert lib.cp_attn_fwd_host(uly._h, r(q), r(k), r(k), r(o), r(lse), None, 0, None) == binding.CP_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_tensors_in_the_wrong_memory():
+    # a host tensor handed to a kernel would be a GPU memory fault: refused before any call
+    import torch
+    q = torch.zeros((1, 2, 64, 64), dtype=torch.bfloat16)
+    plan = Plan(1, 2, 2, 64, 64, n_cp=2)
+    with pytest.raises(ValueError):
+        plan.fwd(q, q, q)
+    with pytest.raises(ValueError):
+        plan.ring_step(0, 0, q, q, q)
+    with pytest.raises(ValueError):
+        binding.lse_merge(q.float(), q[:, :, :, 0].float(), q.float(), q[:, :, :, 0].float())
+    with pytest.raises(ValueError):
+        binding.seq2head(2, q)
+    x = torch.zeros((1, 2, 256), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.ConvPlan(1, 2, 256, 5, 2).fwd(x, torch.zeros((2, 5), dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        binding.FftConvPlan(1, 2, 256, 2).fwd(x, torch.zeros((2, 256), dtype=torch.bfloat16))
