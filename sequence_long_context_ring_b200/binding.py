@@ -143,11 +143,29 @@ def _stream(stream) -> Optional[int]:
 
 
 def _on_device(*tensors) -> None:
-    """The device entry points dereference their pointers in kernels: a host tensor there would
-    be a GPU memory fault, so it is refused before the call."""
+    """The device entry points dereference their pointers in kernels launched on the current
+    device: a host tensor, or one on another GPU, would be a memory fault there, so it is
+    refused before the call."""
+    cur = None
     for t in tensors:
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise ValueError("expected a CUDA tensor (this call's kernels read and write device memory)")
+        if cur is None:
+            cur = torch.cuda.current_device()
+        if t.device.index != cur:
+            raise ValueError(f"tensor on {t.device}, but the kernels launch on cuda:{cur} "
+                             "(select the tensor's device first)")
+
+
+def _ws_args(ws):
+    """(pointer, size in bytes) of a workspace tensor, or (None, 0) without one."""
+    if ws is None:
+        return None, 0
+    if not ws.is_contiguous():
+        raise ValueError("the workspace must be contiguous")
+    return ws.data_ptr(), ws.numel() * ws.element_size()
 
 
 def _on_host(*tensors) -> None:
@@ -213,8 +231,7 @@ class Plan:
             lse = torch.empty((c.B, c.Hq, c.L), dtype=torch.float32, device=q.device)
         if ws is None:
             ws = self.workspace(False, q.device)
-        wptr = ws.data_ptr() if ws is not None else None
-        wlen = ws.numel() if ws is not None else 0
+        wptr, wlen = _ws_args(ws)
         td = [tensor_desc(t) for t in (q, k, v, o, lse)]
         _check(lib().cp_attn_fwd(self._h, *[ctypes.byref(t) for t in td], wptr, wlen, _stream(stream)),
                "cp_attn_fwd")
@@ -234,8 +251,8 @@ class Plan:
         if ws is None:
             ws = torch.empty(self.host_workspace_size(), dtype=torch.uint8, device="cuda")
         td = [tensor_desc(t) for t in (q, k, v, o, lse)]
-        _check(lib().cp_attn_fwd_host(self._h, *[ctypes.byref(t) for t in td], ws.data_ptr(), ws.numel(),
-                                      _stream(stream)), "cp_attn_fwd_host")
+        _check(lib().cp_attn_fwd_host(self._h, *[ctypes.byref(t) for t in td], *_ws_args(ws), _stream(stream)),
+               "cp_attn_fwd_host")
         return o, lse
 
     def fwd_noalloc(self, q, k, v, o, lse, stream=None):
@@ -256,8 +273,7 @@ class Plan:
         dv = torch.empty_like(v) if dv is None else dv
         if ws is None:
             ws = self.workspace(True, q.device)
-        wptr = ws.data_ptr() if ws is not None else None
-        wlen = ws.numel() if ws is not None else 0
+        wptr, wlen = _ws_args(ws)
         td = [tensor_desc(t) for t in (q, k, v, o, lse, dout, dq, dk, dv)]
         _check(lib().cp_attn_bwd(self._h, *[ctypes.byref(t) for t in td], wptr, wlen, _stream(stream)),
                "cp_attn_bwd")
@@ -404,6 +420,6 @@ class FftConvPlan:
         y = torch.empty_like(x) if y is None else y
         ws = self.workspace(x.device) if ws is None else ws
         td = [tensor_desc(t) for t in (x, h, y)]
-        _check(lib().cp_fftconv_fwd(self._h, *[ctypes.byref(t) for t in td], ws.data_ptr(), ws.numel(),
-                                    _stream(stream)), "cp_fftconv_fwd")
+        _check(lib().cp_fftconv_fwd(self._h, *[ctypes.byref(t) for t in td], *_ws_args(ws), _stream(stream)),
+               "cp_fftconv_fwd")
         return y

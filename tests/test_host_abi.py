@@ -243,3 +243,26 @@ def test_binding_refuses_tensors_in_the_wrong_memory():
         binding.ConvPlan(1, 2, 256, 5, 2).fwd(x, torch.zeros((2, 5), dtype=torch.bfloat16))
     with pytest.raises(ValueError):
         binding.FftConvPlan(1, 2, 256, 2).fwd(x, torch.zeros((2, 256), dtype=torch.bfloat16))
+
+
+def test_binding_refuses_a_tensor_on_another_gpu(monkeypatch):
+    # the kernels launch on the current device: a tensor on another GPU is refused before any
+    # call (stand-in tensors, so no GPU is needed)
+    import types
+
+    import torch
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    on0 = types.SimpleNamespace(is_cuda=True, device=torch.device("cuda", 0))
+    on1 = types.SimpleNamespace(is_cuda=True, device=torch.device("cuda", 1))
+    binding._on_device(on0, None, on0)
+    with pytest.raises(ValueError, match="cuda:1"):
+        binding._on_device(on0, on1)
+
+
+def test_workspace_size_is_counted_in_bytes():
+    import torch
+    assert binding._ws_args(None) == (None, 0)
+    ws = torch.empty(10, dtype=torch.float32)
+    assert binding._ws_args(ws) == (ws.data_ptr(), 40)
+    with pytest.raises(ValueError):
+        binding._ws_args(torch.empty((4, 4), dtype=torch.uint8)[:, ::2])
