@@ -78,6 +78,7 @@ def _rank(rank, world, port, causal, split, out):
     (1, True, "contiguous"), (2, True, "contiguous"), (3, True, "contiguous"), (4, True, "contiguous"),
     (1, False, "contiguous"), (3, False, "contiguous"),
     (2, True, "zigzag"), (3, True, "zigzag"), (4, True, "zigzag"), (3, True, "striped"), (2, False, "zigzag"),
+    (8, True, "zigzag"), (6, False, "striped"), (5, True, "contiguous"),
 ])
 def test_ring_across_processes_equals_full_attention(world, causal, split):
     import oracle
