@@ -172,3 +172,51 @@ def test_rings_in_process_subgroups():
         c = q.shape[2] // 2
         np.testing.assert_allclose(res[rank][0], o_ref[:, :, gr * c:(gr + 1) * c], atol=1e-12)
         np.testing.assert_allclose(res[rank][1], l_ref[:, :, gr * c:(gr + 1) * c], atol=1e-12)
+
+
+def _rank_failure(rank, world, port, mode, out):
+    import datetime
+    import time
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from sequence_long_context_ring_b200 import ring_dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=2))
+    if rank == 1:
+        # the failing peer: it leaves before its first exchange, or stalls past the timeout
+        out[rank] = mode
+        if mode == "stalls":
+            time.sleep(5)
+        dist.destroy_process_group()
+        return
+    q = torch.zeros((1, 2, 4, 8), dtype=torch.float64)
+    zeros = lambda qq, kk, vv, diag, scale: (torch.zeros_like(qq), torch.zeros(qq.shape[:3], dtype=qq.dtype))
+    t0 = time.time()
+    try:
+        ring_dist.ring_attention(q, q[:, :1], q[:, :1], partial_fn=zeros, merge_fn=lambda *a: None)
+        out[rank] = ("returned", time.time() - t0)
+    except RuntimeError:
+        out[rank] = ("raised", time.time() - t0)
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:
+            pass
+
+
+@pytest.mark.parametrize("mode", ["leaves", "stalls"])
+def test_a_failing_peer_ends_the_ring_with_an_error(mode):
+    # failure detection on the host: the surviving rank's exchange raises (connection closed,
+    # or the process group's 2 s timeout) instead of waiting for ever
+    port = 29750 + (os.getpid() * 13 + len(mode)) % 2000
+    with mp.get_context("spawn").Manager() as man:
+        out = man.dict()
+        mp.spawn(_rank_failure, args=(2, port, mode, out), nprocs=2, join=True)
+        res = dict(out)
+    assert res[1] == mode
+    outcome, seconds = res[0]
+    assert outcome == "raised"
+    assert seconds < 4.5
