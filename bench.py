@@ -122,17 +122,24 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
+        return self.summarize(self.lines)
+
+    @staticmethod
+    def summarize(lines):
+        """Median SM clock, max clock and the throttle reasons seen active, from the sampled
+        CSV lines (sm, max, power, active mask, hw_slowdown, hw_thermal, sw_thermal, sw_power_cap)."""
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in lines:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 8:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
+                clk, clk_max = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
+            sm.append(clk)
+            mx = clk_max
             for nm, val in zip(names, parts[4:8]):
                 if val.lower() == "active":
                     reasons.add(nm)

@@ -36,3 +36,20 @@ def test_reference_arm_other_ranks_exit_quietly():
     res = _run({"RANK": "1"})
     assert res.returncode == 0, res.stderr
     assert res.stdout.strip() == ""
+
+
+def test_clock_summary_reports_median_max_and_active_reasons():
+    sys.path.insert(0, ROOT)
+    import bench
+    lines = [
+        "1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "1800, 1965, 990.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "1700, 1965, 995.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "[N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",   # unreadable sample
+        "short line",
+    ]
+    s = bench.ClockSampler.summarize(lines)
+    assert s == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    hot = lines[:1] + ["1200, 1965, 800, 0x8, Active, Not Active, Active, Not Active"]
+    assert bench.ClockSampler.summarize(hot)["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert bench.ClockSampler.summarize([]) is None
