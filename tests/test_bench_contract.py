@@ -53,3 +53,13 @@ def test_clock_summary_reports_median_max_and_active_reasons():
     hot = lines[:1] + ["1200, 1965, 800, 0x8, Active, Not Active, Active, Not Active"]
     assert bench.ClockSampler.summarize(hot)["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     assert bench.ClockSampler.summarize([]) is None
+
+
+def test_traffic_figure_is_dropped_once_the_kernel_changes(monkeypatch):
+    # the committed DRAM bytes per launch belong to one version of the forward kernel's source
+    sys.path.insert(0, ROOT)
+    import bench
+    w = "c3_llama3_8b_gqa_L212992_N16"
+    assert bench.traffic_from_profile(w) is not None
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
+    assert bench.traffic_from_profile(w) is None
