@@ -60,6 +60,9 @@ def test_traffic_figure_is_dropped_once_the_kernel_changes(monkeypatch):
     sys.path.insert(0, ROOT)
     import bench
     w = "c3_llama3_8b_gqa_L212992_N16"
-    assert bench.traffic_from_profile(w) is not None
+    with open(os.path.join(ROOT, "profiles", "ring_fwd_kernel_traffic.json")) as f:
+        rec = json.load(f)
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: rec["kernel_source_hash"])
+    assert bench.traffic_from_profile(w) == rec["per_launch_bytes"][w]
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
     assert bench.traffic_from_profile(w) is None
