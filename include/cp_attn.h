@@ -152,12 +152,14 @@ cp_status_t cp_attn_bwd(const cp_plan_t* plan, const cp_tensor_t* q, const cp_te
  * that loads the library holds those 64 MiB until the process exits.  Problems whose forward
  * workspace (cp_attn_workspace_size) exceeds 64 MiB are rejected with CP_ERR_WORKSPACE before
  * any launch.  The library calls no allocating routine here.  The first call on a device looks
- * up the scratch's device address (cudaGetSymbolAddress, once per device); make that first
- * call before any stream capture.  All calls share the one scratch array: calls whose GPU
+ * up the scratch's device address (cudaGetSymbolAddress) and caches it for the rest of the
+ * process, per device ordinal, so a cudaDeviceReset afterwards leaves a stale address; make
+ * that first call before any stream capture.  All calls share the one scratch array: calls whose GPU
  * work overlaps (on different streams, or from different threads) race on it and must be
  * serialised by the caller.  The scratch keeps the last call's contents; every byte a call
  * reads is written earlier in the same call.  Device-side wait expiries are not recorded
- * (there is no status word without an allocation); the waits stay bounded. */
+ * (there is no status word without an allocation); the waits stay bounded.  For the same
+ * reason a plan with debug_fault set gets CP_ERR_UNSUPPORTED before any launch. */
 cp_status_t cp_attn_fwd_noalloc(const cp_plan_t* plan, const cp_tensor_t* q, const cp_tensor_t* k,
                                 const cp_tensor_t* v, cp_tensor_t* o, cp_tensor_t* lse, void* stream);
 

@@ -934,7 +934,8 @@ constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
 
-// Device address of the static scratch on the current device (looked up once per device).
+// Device address of the static scratch on the current device, looked up once per process and
+// device ordinal and cached from then on (a cudaDeviceReset would invalidate it).
 cp_status_t noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return CP_ERR_CUDA;
@@ -956,6 +957,9 @@ extern "C" cp_status_t cp_attn_fwd_noalloc(const cp_plan_t* plan, const cp_tenso
   if (!plan) return CP_ERR_INVALID_ARG;
   const cp_attn_config_t& c = plan->cfg;
   if (c.mode != CP_MODE_ULYSSES && c.mode != CP_MODE_2D) return CP_ERR_INVALID_ARG;
+  // This path has no status word, so an injected wait expiry could not be reported: each CTA
+  // would wait out its full limit and the call would return CP_OK with O/LSE unwritten.
+  if (c.debug_fault != 0) return CP_ERR_UNSUPPORTED;
   CP_TRY(check3(lse, c.B, c.Hq, c.L));
   CP_TRY(check4(q, CP_BF16, c.B, c.L, c.Hq, c.d));
   CP_TRY(check4(k, CP_BF16, c.B, c.L, c.Hkv, c.d));

@@ -266,3 +266,13 @@ def test_workspace_size_is_counted_in_bytes():
     assert binding._ws_args(ws) == (ws.data_ptr(), 40)
     with pytest.raises(ValueError):
         binding._ws_args(torch.empty((4, 4), dtype=torch.uint8)[:, ::2])
+
+
+def test_noalloc_forward_refuses_fault_injection_before_any_launch():
+    # the allocation-free forward has no status word to report an injected wait expiry, so a
+    # plan with debug_fault set is refused before the tensors are even looked at
+    lib = binding.lib()
+    plan = Plan(1, 8, 8, 512, 64, n_cp=4, mode="ulysses", debug_fault=1)
+    assert lib.cp_attn_fwd_noalloc(plan._h, None, None, None, None, None, None) == binding.CP_ERR_UNSUPPORTED
+    ring = Plan(1, 8, 8, 512, 64, n_cp=4, debug_fault=1)
+    assert lib.cp_attn_fwd_noalloc(ring._h, None, None, None, None, None, None) == binding.CP_ERR_INVALID_ARG

@@ -19,6 +19,24 @@ def test_zigzag_matches_the_pages_worked_example():
     assert got == g["shards_per_rank"]
 
 
+def test_striped_matches_the_fixture_of_its_reading():
+    g = json.load(open(os.path.join(HERE, "golden", "striped_shards_n4.json")))
+    n = g["n_cp"]
+    assert [list(sp.shards_of_rank("striped", n, r)) for r in range(n)] == g["shards_per_rank"]
+    assert [sp.rank_positions("striped", n, g["L"], r).tolist() for r in range(n)] == g["positions_per_rank"]
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 8])
+def test_striped_deals_shards_round_robin(n):
+    # stripes: walking the shards in sequence order, the ranks take turns, so shard s belongs
+    # to rank s mod N (any other permutation of shards would break this for some n)
+    owner = {}
+    for r in range(n):
+        for s in sp.shards_of_rank("striped", n, r):
+            owner[s] = r
+    assert [owner[s] for s in range(2 * n)] == [s % n for s in range(2 * n)]
+
+
 @pytest.mark.parametrize("split", sp.SPLITS)
 @pytest.mark.parametrize("n,L", [(1, 8), (2, 8), (3, 12), (4, 32), (5, 40)])
 def test_every_position_belongs_to_exactly_one_rank(split, n, L):
