@@ -8,17 +8,20 @@ namespace cpattn {
 
 // ---- Ulysses all-to-all on one GPU -------------------------------------------------------
 // Swaps axes 1 and 2 of a [B, X, Y, d] view: out[b, y, x, :] = in[b, x, y, :].  Rows of d
-// elements are contiguous on both sides, so the copy moves whole 16-byte vectors: thread
-// groups walk the OUTPUT in order (fully sequential writes) and read 16-byte pieces of
-// 2*d-byte rows (d = 128 -> 256-byte contiguous reads).  Each thread moves kVecPerThread
-// vectors spaced one block apart, so every load of a warp is coalesced and several loads
-// per thread are in flight.  ("05. 長系列の分散学習（Context Parallelism）" §2: the
-// re-layout [D, L/N_cp] -> [H/N_cp, L]; "Ulyssesシーケンス並列化の核心" steps 2 and 4.)
+// elements are contiguous on both sides, so the copy moves whole 16-byte vectors.  A block
+// owns a run of consecutive OUTPUT rows (fully sequential writes): it first resolves each row's
+// source and destination offsets once (the only divisions, and the split's rank-row map, run
+// per row, not per vector), then every thread moves up to kPermVecPerThread vectors whose loads
+// are all issued before the first store, so several reads per thread are in flight.
+// ("05. 長系列の分散学習（Context Parallelism）" §2: the re-layout [D, L/N_cp] -> [H/N_cp, L];
+// "Ulyssesシーケンス並列化の核心" steps 2 and 4.)
 struct PermuteParams {
   const uint4* in;
   uint4* out;
-  long long n_vec;       // total 16-byte vectors
+  long long n_rows;      // B * Y * X output rows
   int vec_per_row;       // d * elem_bytes / 16
+  int vec_shift;         // log2(vec_per_row) when it is a power of two, else -1
+  int rows_per_block;    // output rows per block (<= kPermMaxRows)
   int X, Y;              // in is [B, X, Y, row]; out is [B, Y, X, row]
   long long in_sb, in_sx, in_sy;     // strides in 16-byte vectors
   long long out_sb, out_sy, out_sx;
@@ -50,38 +53,64 @@ __device__ __forceinline__ int pos_of_rank_row(const PermuteParams& p, int u) {
 }
 
 constexpr int kPermThreads = 256;
-constexpr int kVecPerThread = 4;
+constexpr int kPermVecPerThread = 4;                                  // per pass of the block
+constexpr int kPermVecPerPass = kPermThreads * kPermVecPerThread;     // 1024 vectors (16 KB)
+constexpr int kPermMaxRows = 256;
 
 __global__ void __launch_bounds__(kPermThreads) permute_rows_kernel(const PermuteParams p) {
-  const long long base = static_cast<long long>(blockIdx.x) * (kPermThreads * kVecPerThread) + threadIdx.x;
-  uint4 v[kVecPerThread];
-  long long dst[kVecPerThread];
-#pragma unroll
-  for (int u = 0; u < kVecPerThread; ++u) {
-    const long long g = base + u * kPermThreads;  // index in output order (b, y, x, vec)
-    dst[u] = -1;
-    if (g < p.n_vec) {
-      long long t = g;
-      const int vec = static_cast<int>(t % p.vec_per_row);
-      t /= p.vec_per_row;
-      const int x = static_cast<int>(t % p.X);
-      t /= p.X;
-      const int y = static_cast<int>(t % p.Y);
-      const long long b = t / p.Y;
+  __shared__ long long src_row[kPermMaxRows];
+  __shared__ long long dst_row[kPermMaxRows];
+  const long long row0 = static_cast<long long>(blockIdx.x) * p.rows_per_block;
+  for (int r = threadIdx.x; r < p.rows_per_block; r += kPermThreads) {
+    const long long R = row0 + r;   // output row in (b, y, x) order
+    long long src = -1, dst = -1;
+    if (R < p.n_rows) {
+      const long long by = R / p.X;
+      const int x = static_cast<int>(R - by * p.X);
+      const long long b = by / p.Y;
+      const int y = static_cast<int>(by - b * p.Y);
       const int xi = p.remap == 1 ? rank_row_of_pos(p, x) : x;
       const int yi = p.remap == 2 ? pos_of_rank_row(p, y) : y;
-      v[u] = __ldg(p.in + b * p.in_sb + xi * p.in_sx + yi * p.in_sy + vec);
-      dst[u] = b * p.out_sb + y * p.out_sy + x * p.out_sx + vec;
+      src = b * p.in_sb + xi * p.in_sx + yi * p.in_sy;
+      dst = b * p.out_sb + y * p.out_sy + x * p.out_sx;
     }
+    src_row[r] = src;
+    dst_row[r] = dst;
   }
+  __syncthreads();
+  const int total = p.rows_per_block * p.vec_per_row;
+  for (int base = 0; base < total; base += kPermVecPerPass) {
+    uint4 v[kPermVecPerThread];
+    long long dst[kPermVecPerThread];
 #pragma unroll
-  for (int u = 0; u < kVecPerThread; ++u)
-    if (dst[u] >= 0) p.out[dst[u]] = v[u];
+    for (int u = 0; u < kPermVecPerThread; ++u) {
+      const int g = base + u * kPermThreads + static_cast<int>(threadIdx.x);
+      dst[u] = -1;
+      if (g < total) {
+        const int r = p.vec_shift >= 0 ? (g >> p.vec_shift) : g / p.vec_per_row;
+        const int vec = g - r * p.vec_per_row;
+        const long long src = src_row[r];
+        if (src >= 0) {
+          v[u] = __ldg(p.in + src + vec);
+          dst[u] = dst_row[r] + vec;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPermVecPerThread; ++u)
+      if (dst[u] >= 0) p.out[dst[u]] = v[u];
+  }
 }
 
 // ---- step-wise LSE merge ----------------------------------------------------------------
 // (O_acc, LSE_acc) <- (O_acc, LSE_acc) (+) (O_part, LSE_part) in place ("ring attention:
-// key/value をリングで回す" step 3).  One row of d fp32 per d/4 lanes (16-byte vectors).
+// key/value をリングで回す" step 3):  m = max(l, l'); w = e^(l - m), w' = e^(l' - m);
+// O <- (w O + w' O') / (w + w');  l <- m + ln(w + w').  A row of d fp32 is d/4 lanes of 16-byte
+// vectors (32 lanes at d = 128, 16 at d = 64).  The grid is (row blocks, (b, h) pairs, strided
+// over B * H): a block takes kMergeSlots * 32 / (d/4) rows per warp of one (b, h), and each lane
+// issues all its loads (kMergeSlots rows of O, O' and the two LSE values) before the
+// arithmetic, so no index division runs per element and several 16-byte reads per lane are in
+// flight.
 struct MergeParams {
   float* o_acc;
   float* lse_acc;
@@ -92,42 +121,58 @@ struct MergeParams {
   long long op_sb, op_sh, op_sr, lp_sb, lp_sh, lp_sr;
 };
 
-__global__ void __launch_bounds__(256) lse_merge_kernel(const MergeParams p) {
-  const int lanes_per_row = p.d / 4;  // 16 or 32: a row never straddles two warps
-  const long long gthread = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long row = gthread / lanes_per_row;
-  const int vec = static_cast<int>(gthread % lanes_per_row);
-  const long long n_rows = static_cast<long long>(p.B) * p.H * p.R;
-  const bool live = row < n_rows;
-  float* la = nullptr;
-  float lse_out = -INFINITY;
-  if (live) {
-    const int r = static_cast<int>(row % p.R);
-    const int h = static_cast<int>((row / p.R) % p.H);
-    const int b = static_cast<int>(row / (static_cast<long long>(p.R) * p.H));
-    la = p.lse_acc + b * p.la_sb + h * p.la_sh + r * p.la_sr;
-    const float lb = p.lse_part[b * p.lp_sb + h * p.lp_sh + r * p.lp_sr];
-    const float l0 = *la;
-    const float m = fmaxf(l0, lb);
-    float4* oa = reinterpret_cast<float4*>(p.o_acc + b * p.oa_sb + h * p.oa_sh + r * p.oa_sr) + vec;
-    const float4 ob = reinterpret_cast<const float4*>(p.o_part + b * p.op_sb + h * p.op_sh + r * p.op_sr)[vec];
-    float4 out;
-    if (m == -INFINITY) {
-      out = make_float4(0.f, 0.f, 0.f, 0.f);
-    } else {
-      const float wa = (l0 == -INFINITY) ? 0.f : expf(l0 - m);
-      const float wb = (lb == -INFINITY) ? 0.f : expf(lb - m);
-      const float inv = 1.f / (wa + wb);
-      const float ca = wa * inv, cb = wb * inv;
-      const float4 a = *oa;
-      out = make_float4(ca * a.x + cb * ob.x, ca * a.y + cb * ob.y, ca * a.z + cb * ob.z, ca * a.w + cb * ob.w);
-      lse_out = m + logf(wa + wb);
+constexpr int kMergeThreads = 256;
+constexpr int kMergeSlots = 4;     // rows (per 32/(d/4) lanes) a lane handles in one pass
+
+__global__ void __launch_bounds__(kMergeThreads) lse_merge_kernel(const MergeParams p) {
+  const int lpr = p.d >> 2;                       // lanes per row: 16 or 32
+  const int rows_per_slot = 32 / lpr;             // rows a warp covers per slot: 2 or 1
+  const int rows_per_warp = rows_per_slot * kMergeSlots;
+  const int rows_per_block = rows_per_warp * (kMergeThreads / 32);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int vec = lane & (lpr - 1);
+  const int r0 = blockIdx.x * rows_per_block + warp * rows_per_warp + lane / lpr;
+  for (int bh = blockIdx.y; bh < p.B * p.H; bh += gridDim.y) {
+  const int b = bh / p.H, h = bh - b * p.H;
+  float* oa_base = p.o_acc + b * p.oa_sb + h * p.oa_sh;
+  const float* op_base = p.o_part + b * p.op_sb + h * p.op_sh;
+  float* la_base = p.lse_acc + b * p.la_sb + h * p.la_sh;
+  const float* lp_base = p.lse_part + b * p.lp_sb + h * p.lp_sh;
+  float4 a[kMergeSlots], o[kMergeSlots];
+  float l0[kMergeSlots], l1[kMergeSlots];
+#pragma unroll
+  for (int k = 0; k < kMergeSlots; ++k) {
+    const int r = r0 + k * rows_per_slot;
+    if (r < p.R) {
+      a[k] = reinterpret_cast<const float4*>(oa_base + r * p.oa_sr)[vec];
+      o[k] = __ldg(reinterpret_cast<const float4*>(op_base + r * p.op_sr) + vec);
+      l0[k] = la_base[r * p.la_sr];
+      l1[k] = __ldg(lp_base + r * p.lp_sr);
     }
-    *oa = out;
   }
-  // every lane of a row has read *la before its first lane overwrites it
+  // every lane of a row has read its LSE before the row's first lane overwrites it
   __syncwarp();
-  if (live && vec == 0) *la = lse_out;
+#pragma unroll
+  for (int k = 0; k < kMergeSlots; ++k) {
+    const int r = r0 + k * rows_per_slot;
+    if (r < p.R) {
+      const float m = fmaxf(l0[k], l1[k]);
+      float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
+      float lse = -INFINITY;
+      if (m != -INFINITY) {
+        // one weight is 1; an empty side (LSE = -inf) gets weight 0
+        const float wa = __expf(l0[k] - m), wb = __expf(l1[k] - m);
+        const float inv = __frcp_rn(wa + wb);
+        const float ca = wa * inv, cb = wb * inv;
+        out = make_float4(ca * a[k].x + cb * o[k].x, ca * a[k].y + cb * o[k].y, ca * a[k].z + cb * o[k].z,
+                          ca * a[k].w + cb * o[k].w);
+        lse = m + __logf(wa + wb);
+      }
+      reinterpret_cast<float4*>(oa_base + r * p.oa_sr)[vec] = out;
+      if (vec == 0) la_base[r * p.la_sr] = lse;
+    }
+  }
+  }
 }
 
 // ---- backward preprocess: D_i = sum_e dO_ie * O_ie ------------------------------------------
