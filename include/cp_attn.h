@@ -98,10 +98,13 @@ typedef struct {
   cp_split_t split;
   float softmax_scale;  /* 0 => 1/sqrt(d)                                                       */
   uint64_t wait_limit_ns; /* bound of every device-side wait; 0 => 2 s                          */
-  int debug_fault;      /* 0 in production.  1 => the forward kernel's load warp skips the
-                           query-tile load, so every consumer's bounded wait expires and the
-                           kernel ends with CP_ERR_TIMEOUT in the status word (a test of the
-                           timeout path; nothing faults or hangs).                              */
+  int debug_fault;      /* 0 in production.  A test of the timeout path, where one load warp
+                           leaves out a load so that every consumer's bounded wait expires and
+                           the kernel ends with CP_ERR_TIMEOUT in the status word (nothing
+                           faults or hangs): 1 => the forward kernel skips the query-tile load;
+                           2 => the backward's dK/dV kernel skips the K/V tile load; 3 => the
+                           backward's dQ kernel skips the Q/dO tile load.  Other values:
+                           CP_ERR_INVALID_ARG.                                                  */
 } cp_attn_config_t;
 
 typedef struct cp_plan cp_plan_t;
@@ -168,7 +171,9 @@ cp_status_t cp_attn_fwd_noalloc(const cp_plan_t* plan, const cp_tensor_t* q, con
  * works but its copies do not overlap the kernels).  The library copies the inputs in, runs
  * the same forward kernel, and copies O and LSE out, pipelined over blocks of KV heads: while
  * one block computes on `stream`, the next block's Q/K/V arrive and the previous block's O/LSE
- * leave on two internal streams (GQA blocks are independent problems, so the result is
+ * leave on two copy streams (created with their events at the plan's first such call on a
+ * device and kept until cp_attn_plan_destroy; calls on one plan enqueue one at a time, so the
+ * plan stays shareable between threads) (GQA blocks are independent problems, so the result is
  * bit-identical to cp_attn_fwd).  Device staging for all five tensors comes from `ws`, a
  * device buffer of at least cp_attn_host_workspace_size bytes, 256-byte aligned.  Everything
  * is enqueued behind the work already on `stream`; the host buffers are complete, and `ws`

@@ -37,6 +37,10 @@ typedef struct {
   int n_cp;               /* virtual ranks holding contiguous shards of c = L / n_cp samples;
                              L % n_cp == 0 and l_h - 1 <= c                                    */
   uint64_t wait_limit_ns; /* bound of every device-side wait; 0 => 2 s                          */
+  int debug_fault;        /* 0 in production.  1 => the tensor-core kernel's load warp leaves out
+                             its first tile's load, so the bounded waits expire and the call's
+                             status word reads CP_ERR_TIMEOUT (a test of the timeout path;
+                             nothing faults or hangs).  Other values: CP_ERR_INVALID_ARG.       */
 } cp_conv_config_t;
 
 typedef struct cp_conv_plan cp_conv_plan_t;

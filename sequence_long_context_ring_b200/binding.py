@@ -43,7 +43,7 @@ class CpConfig(ctypes.Structure):
 
 class ConvConfig(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("D", ctypes.c_int), ("L", ctypes.c_int), ("lh", ctypes.c_int),
-                ("n_cp", ctypes.c_int), ("wait_limit_ns", ctypes.c_uint64)]
+                ("n_cp", ctypes.c_int), ("wait_limit_ns", ctypes.c_uint64), ("debug_fault", ctypes.c_int)]
 
 
 class FftConvConfig(ctypes.Structure):
@@ -342,8 +342,9 @@ class ConvPlan:
     """A cp_conv plan: the causal depthwise FIR convolution of a sequence sharded over n_cp
     contiguous virtual ranks (include/cp_conv.h)."""
 
-    def __init__(self, B: int, D: int, L: int, lh: int, n_cp: int = 1, wait_limit_ns: int = 0):
-        self.cfg = ConvConfig(B, D, L, lh, n_cp, int(wait_limit_ns))
+    def __init__(self, B: int, D: int, L: int, lh: int, n_cp: int = 1, wait_limit_ns: int = 0,
+                 debug_fault: int = 0):
+        self.cfg = ConvConfig(B, D, L, lh, n_cp, int(wait_limit_ns), int(debug_fault))
         h = ctypes.c_void_p()
         _check(lib().cp_conv_plan(ctypes.byref(self.cfg), ctypes.byref(h)), "cp_conv_plan")
         self._h = h

@@ -54,6 +54,7 @@ struct DqParams {
   long long dq_sb, dq_sh, dq_sl;
   int* status;
   unsigned long long wait_limit_ns;
+  int debug_fault;    // 3: the load warp skips the Q/dO tile load (a test of the timeout path)
 };
 
 struct DqItem {
@@ -202,11 +203,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       tma_prefetch_desc(&tm_do);
       const uint64_t pol_kv = policy_evict_last();
       const uint64_t pol_q = policy_evict_first();
-      mbar_arrive_expect_tx(q_full, 2 * kTile);
+      const bool load_q = (p.debug_fault != 3);
+      if (load_q) {
+        mbar_arrive_expect_tx(q_full, 2 * kTile);
 #pragma unroll
-      for (int x = 0; x < kBoxes; ++x) {
-        tma_load_4d(q_s + x * kBoxBytes, &tm_q, q_full, x * 64, it.row0, it.h, it.b, pol_q);
-        tma_load_4d(do_s + x * kBoxBytes, &tm_do, q_full, x * 64, it.row0, it.h, it.b, pol_q);
+        for (int x = 0; x < kBoxes; ++x) {
+          tma_load_4d(q_s + x * kBoxBytes, &tm_q, q_full, x * 64, it.row0, it.h, it.b, pol_q);
+          tma_load_4d(do_s + x * kBoxBytes, &tm_do, q_full, x * 64, it.row0, it.h, it.b, pol_q);
+        }
       }
       int nk = 0, nv = 0;  // loads issued
       DqKvIter kvi(p, it);
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
       }
       // drain: every load this thread issued has landed before the CTA can exit
-      dq_wait_drain(q_full, 0, ctl);
+      if (load_q) dq_wait_drain(q_full, 0, ctl);
       for (int n = (nk > kDqKSlots ? nk - kDqKSlots : 0); n < nk; ++n)
         dq_wait_drain(&k_full[n % kDqKSlots], (n / kDqKSlots) & 1, ctl);
       for (int n = (nv > kDqVSlots ? nv - kDqVSlots : 0); n < nv; ++n)

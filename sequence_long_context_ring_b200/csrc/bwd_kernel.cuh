@@ -24,6 +24,11 @@
 // TMEM columns: S^T [0,128)  dP^T [128,256)  dV [256,384)  dK [384,512).  P^T (bf16, two per
 // column) of query columns [64h, 64h+64) is written over S^T columns [64h, 64h+32), which
 // that warpgroup has already read; dS^T likewise over dP^T.
+// MMA order per query tile i: dV(i), S^T(i+1), dK(i), dP^T(i+1).  S^T(i+1) may overwrite the
+// S^T columns as soon as dV(i) has been issued (the tensor pipe runs one thread's MMAs in
+// order), so the warps compute P(i+1) while the tensor cores run dK(i) and dP^T(i+1).
+// Shared memory holds, per Q/dO stage, -LSE * log2(e) and D of the tile's 128 queries: the
+// warps read them as broadcast 16-byte vectors.
 #pragma once
 #include <cstddef>
 #include "sm100.cuh"
@@ -59,6 +64,7 @@ struct BwdParams {
   long long dv_sb, dv_sh, dv_sl;
   int* status;
   unsigned long long wait_limit_ns;
+  int debug_fault;    // 2: the load warp skips the K/V tile load (a test of the timeout path)
 };
 
 struct BwdItem {
@@ -204,16 +210,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == kBwdLoadWarp) {
     // ---------------- loads ----------------
     const uint64_t pol_keep = policy_evict_last();
+    const bool load_kv = (p.debug_fault != 2);
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(kv_full, 2 * kTile);
+      if (load_kv) {
+        mbar_arrive_expect_tx(kv_full, 2 * kTile);
 #pragma unroll
-      for (int x = 0; x < kBoxes; ++x) {
-        tma_load_4d(k_s + x * kBoxBytes, &tm_k, kv_full, x * 64, it.kv0, it.g, it.b, pol_keep);
-        tma_load_4d(v_s + x * kBoxBytes, &tm_v, kv_full, x * 64, it.kv0, it.g, it.b, pol_keep);
+        for (int x = 0; x < kBoxes; ++x) {
+          tma_load_4d(k_s + x * kBoxBytes, &tm_k, kv_full, x * 64, it.kv0, it.g, it.b, pol_keep);
+          tma_load_4d(v_s + x * kBoxBytes, &tm_v, kv_full, x * 64, it.kv0, it.g, it.b, pol_keep);
+        }
       }
     }
     bool ok = true;
@@ -221,27 +230,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int i = 0; i < it.n_iter && ok; ++i) {
       const int st = i & 1;
       const uint32_t ph = (i >> 1) & 1;
-      ok = __all_sync(0xffffffffu, wait_bounded(&q_empty[st], ph ^ 1, ctl, kBSiteLoadEmpty));
-      if (!ok) break;
       int h, q0, q_end;
       bwd_qtile(p, it, i, h, q0, q_end);
-      // LSE (log2 units) and D of the tile's 128 query rows; rows outside the chunk get
-      // LSE = +inf (probability 0) so they contribute nothing.
-      float* lse2 = stat_s + st * 256;
-      float* dvec = lse2 + 128;
+      // -LSE (log2 units) and D of the tile's 128 query rows, fetched before the stage is free
+      // (the loads' latency overlaps the wait); rows outside the chunk get -LSE = -inf
+      // (probability 0) and D = 0, so they contribute nothing.
+      float4 nl, dd4;
+      {
+        float l[4], dd[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int rr = lane * 4 + u;
-        const int q = q0 + rr;
-        float l2 = INFINITY, dd = 0.f;
-        if (q < q_end) {
-          l2 = p.lse[it.b * p.lse_sb + h * p.lse_sh + static_cast<long long>(q) * p.lse_sl] *
-               1.4426950408889634f;
-          dd = p.Dvec[(static_cast<long long>(it.b) * p.Hq + h) * p.L + q];
+        for (int u = 0; u < 4; ++u) {
+          const int q = q0 + lane * 4 + u;
+          l[u] = -INFINITY;
+          dd[u] = 0.f;
+          if (q < q_end) {
+            l[u] = -p.lse[it.b * p.lse_sb + h * p.lse_sh + static_cast<long long>(q) * p.lse_sl] *
+                   1.4426950408889634f;
+            dd[u] = p.Dvec[(static_cast<long long>(it.b) * p.Hq + h) * p.L + q];
+          }
         }
-        lse2[rr] = l2;
-        dvec[rr] = dd;
+        nl = make_float4(l[0], l[1], l[2], l[3]);
+        dd4 = make_float4(dd[0], dd[1], dd[2], dd[3]);
       }
+      ok = __all_sync(0xffffffffu, wait_bounded(&q_empty[st], ph ^ 1, ctl, kBSiteLoadEmpty));
+      if (!ok) break;
+      reinterpret_cast<float4*>(stat_s + st * 256)[lane] = nl;
+      reinterpret_cast<float4*>(stat_s + st * 256 + 128)[lane] = dd4;
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(&q_full[st], 2 * kTile);  // the arrive also publishes lse2 / D
@@ -254,7 +268,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ++issued;
     }
     if (lane == 0) {
-      bwd_wait_drain(kv_full, 0, ctl);
+      if (load_kv) bwd_wait_drain(kv_full, 0, ctl);
       for (int s2 = (issued > 2 ? issued - 2 : 0); s2 < issued; ++s2) bwd_wait_drain(&q_full[s2 & 1], (s2 >> 1) & 1, ctl);
     }
     __syncwarp();
@@ -264,41 +278,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr uint32_t idesc_kk = make_idesc_bf16(128, 128, false);     // S^T, dP^T: both K-major
       constexpr uint32_t idesc_tn = make_idesc_bf16(128, D, true);        // dV, dK: A TMEM, B N-major
       const uint32_t k_a = smem_u32(k_s), v_a = smem_u32(v_s);
+      auto q_addr = [&](int i) { return smem_u32(q_s + (i & 1) * kTile); };
+      auto do_addr = [&](int i) { return smem_u32(do_s + (i & 1) * kTile); };
+      // S^T(i) = K Q_i^T and dP^T(i) = V dO_i^T  [M = keys, N = queries, K = d]
+      auto issue_kk = [&](uint32_t d_tmem, uint32_t a, uint32_t b) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          umma_ss(d_tmem, make_sdesc(a + off, 16, 1024), make_sdesc(b + off, 16, 1024), idesc_kk, kk > 0);
+        }
+      };
       bool ok = wait_bounded(kv_full, 0, ctl, kBSiteMmaKV);
+      if (ok && it.n_iter > 0) {
+        ok = wait_bounded(&q_full[0], 0, ctl, kBSiteMmaQ);
+        if (ok) {
+          tc_fence_after();
+          issue_kk(tS, k_a, q_addr(0));
+          umma_commit(s_full);
+          issue_kk(tDP, v_a, do_addr(0));
+          umma_commit(dp_full);
+        }
+      }
       for (int i = 0; i < it.n_iter && ok; ++i) {
         const int st = i & 1;
-        const uint32_t q_a = smem_u32(q_s + st * kTile), do_a = smem_u32(do_s + st * kTile);
-        if (!wait_bounded(&q_full[st], (i >> 1) & 1, ctl, kBSiteMmaQ)) { ok = false; break; }
-        tc_fence_after();
-        // (1) S^T = K Q^T  [M = keys, N = queries, K = d]
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          umma_ss(tS, make_sdesc(k_a + off, 16, 1024), make_sdesc(q_a + off, 16, 1024), idesc_kk, kk > 0);
-        }
-        umma_commit(s_full);
-        // (2) dP^T = V dO^T, over dS^T of the previous tile (its dK MMA was issued before)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          umma_ss(tDP, make_sdesc(v_a + off, 16, 1024), make_sdesc(do_a + off, 16, 1024), idesc_kk, kk > 0);
-        }
-        umma_commit(dp_full);
-        // (3) dV += P^T dO  [A = P^T in TMEM (keys x queries), B = dO N-major]
+        // (1) dV += P^T dO  [A = P^T in TMEM (keys x queries), B = dO N-major]
         if (!wait_bounded(p_full, i & 1, ctl, kBSiteMmaP)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tDV, tS + bwd_a_col(kk), make_sdesc(do_a + kk * 2048, kBoxBytes, 1024), idesc_tn,
+          umma_ts(tDV, tS + bwd_a_col(kk), make_sdesc(do_addr(i) + kk * 2048, kBoxBytes, 1024), idesc_tn,
                   (i > 0 || kk > 0));
-        // (4) dK += dS^T Q  [A = dS^T in TMEM, B = Q N-major]
+        // (2) S^T(i+1) over P^T(i) (read by dV(i), issued before)
+        const bool more = i + 1 < it.n_iter;
+        if (more) {
+          if (!wait_bounded(&q_full[st ^ 1], ((i + 1) >> 1) & 1, ctl, kBSiteMmaQ)) { ok = false; break; }
+          tc_fence_after();
+          issue_kk(tS, k_a, q_addr(i + 1));
+          umma_commit(s_full);
+        }
+        // (3) dK += dS^T Q  [A = dS^T in TMEM, B = Q N-major]; then stage i is free
         if (!wait_bounded(ds_full, i & 1, ctl, kBSiteMmaDs)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tDK, tDP + bwd_a_col(kk), make_sdesc(q_a + kk * 2048, kBoxBytes, 1024), idesc_tn,
+          umma_ts(tDK, tDP + bwd_a_col(kk), make_sdesc(q_addr(i) + kk * 2048, kBoxBytes, 1024), idesc_tn,
                   (i > 0 || kk > 0));
         umma_commit(&q_empty[st]);
+        // (4) dP^T(i+1) over dS^T(i) (read by dK(i), issued before)
+        if (more) {
+          issue_kk(tDP, v_a, do_addr(i + 1));
+          umma_commit(dp_full);
+        }
       }
       if (ok) umma_commit(done_bar);
       umma_commit(drain_bar);
@@ -314,16 +344,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool kv_live = kv_row < it.kv_end;
     const uint32_t lofs = lane_base << 16;
     const uint32_t tSh = tS + lofs + hh * 64, tDPh = tDP + lofs + hh * 64;
-    const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int i = 0; i < it.n_iter; ++i) {
       const int st = i & 1;
       int h, q0, q_end;
       bwd_qtile(p, it, i, h, q0, q_end);
-      const float* lse2 = stat_s + st * 256 + hh * 64;
-      const float* dvec = stat_s + st * 256 + 128 + hh * 64;
-      // causal: query columns c < kv_row - q0 do not see this key (c relative to this half)
+      // -LSE * log2(e) and D of this warpgroup's 64 query columns (broadcast 16-byte reads)
+      const float4* nls4 = reinterpret_cast<const float4*>(stat_s + st * 256 + hh * 64);
+      const float4* dvs4 = reinterpret_cast<const float4*>(stat_s + st * 256 + 128 + hh * 64);
+      // causal: query columns c < kv_row - q0 do not see this key (c relative to this half);
+      // only tiles at the diagonal, and a ragged key tail, need the per-element mask
       const int c_lo = p.causal ? (kv_row - q0 - hh * 64) : 0;
+      const bool masked = __any_sync(0xffffffffu, !kv_live || c_lo > 0);
       if (!__all_sync(0xffffffffu, wait_bounded(s_full, i & 1, ctl, kBSiteSoftS))) { ok = false; break; }
       tc_fence_after();
       uint32_t ra[32], rb[32];
@@ -331,15 +364,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_ld32(tSh + 32, rb);
       tmem_wait_ld();
       uint32_t pk[32];  // P^T of the 64 columns as bf16 pairs, kept for dS
+      // P = 2^(S^T * scale * log2(e) - LSE * log2(e)) for one 32-column chunk, four columns
+      // (two pairs) per -LSE vector
       auto p_chunk = [&](const uint32_t (&r)[32], int cc) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int c = cc * 32 + e;
-          float p0 = ex2_approx(fmaf(__uint_as_float(r[e]), sl2, -lse2[c]));
-          float p1 = ex2_approx(fmaf(__uint_as_float(r[e + 1]), sl2, -lse2[c + 1]));
-          if (!kv_live || c < c_lo) p0 = 0.f;
-          if (!kv_live || c + 1 < c_lo) p1 = 0.f;
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 nl = nls4[cc * 8 + e4];
+          const int e = 4 * e4, c = cc * 32 + e;
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), sl2x2, f2_pack(nl.x, nl.y)), x0,
+                    x1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])), sl2x2, f2_pack(nl.z, nl.w)),
+                    x2, x3);
+          float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+          if (masked) {
+            if (!kv_live || c < c_lo) p0 = 0.f;
+            if (!kv_live || c + 1 < c_lo) p1 = 0.f;
+            if (!kv_live || c + 2 < c_lo) p2 = 0.f;
+            if (!kv_live || c + 3 < c_lo) p3 = 0.f;
+          }
           pk[c >> 1] = pack_bf16x2(p0, p1);
+          pk[(c >> 1) + 1] = pack_bf16x2(p2, p3);
         }
       };
       p_chunk(ra, 0);
@@ -357,14 +402,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_ld32(tDPh + 32, rb);
       tmem_wait_ld();
       uint32_t dsk[32];
+      // dS = P o (dP - D) for one 32-column chunk, four columns per D vector
       auto ds_chunk = [&](const uint32_t (&r)[32], int cc) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int c = cc * 32 + e;
-          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[c >> 1]));
-          const float d0 = pp.x * (__uint_as_float(r[e]) - dvec[c]);
-          const float d1 = pp.y * (__uint_as_float(r[e + 1]) - dvec[c + 1]);
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 dv = dvs4[cc * 8 + e4];
+          const int e = 4 * e4, c = cc * 32 + e;
+          const float2 pa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[c >> 1]));
+          const float2 pb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[(c >> 1) + 1]));
+          const uint64_t da = f2_mul(f2_pack(pa.x, pa.y),
+                                     f2_sub(f2_pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), f2_pack(dv.x, dv.y)));
+          const uint64_t db = f2_mul(f2_pack(pb.x, pb.y), f2_sub(f2_pack(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])),
+                                                                f2_pack(dv.z, dv.w)));
+          float d0, d1, d2, d3;
+          f2_unpack(da, d0, d1);
+          f2_unpack(db, d2, d3);
           dsk[c >> 1] = pack_bf16x2(d0, d1);
+          dsk[(c >> 1) + 1] = pack_bf16x2(d2, d3);
         }
       };
       ds_chunk(ra, 0);

@@ -99,6 +99,7 @@ struct ConvParams {
   long long h_sd;            // channel stride of h (elements)
   int* status;
   unsigned long long wait_limit_ns;
+  int debug_fault;           // 1: the load warp skips its first tile's load (timeout-path test)
 };
 
 // Shared-memory plan.  Three input stages: measured at the full-size workloads, two leave
@@ -205,9 +206,14 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       tma_prefetch_desc(&tm_y);
       const uint64_t pol = policy_evict_first();
       int issued = 0;
+      const int skipped = p.debug_fault == 1 ? 0 : -1;  // tile whose load is left out
       for (int i = 0; i < n_local; ++i) {
         const int s = i % kStages;
         if (i >= kStages && !wait_bounded(&empty[s], ((i / kStages) - 1) & 1, ctl, kCSiteLoad)) break;
+        if (i == skipped) {
+          ++issued;
+          continue;
+        }
         const long long t = t_begin + i;
         const int row = static_cast<int>(t / p.tiles_per_row);
         const int m0 = static_cast<int>(t - static_cast<long long>(row) * p.tiles_per_row) * 128;
@@ -221,7 +227,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       }
       // drain: every load issued has landed before the CTA can exit
       for (int n = (issued > kStages ? issued - kStages : 0); n < issued; ++n)
-        conv_wait_drain(&full[n % kStages], (n / kStages) & 1, ctl);
+        if (n != skipped) conv_wait_drain(&full[n % kStages], (n / kStages) & 1, ctl);
     }
     __syncwarp();
   } else if (warp == 1) {

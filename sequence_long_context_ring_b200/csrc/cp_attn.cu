@@ -5,11 +5,13 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <map>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "aux_kernels.cuh"
 #include "bwd_dq_kernel.cuh"
@@ -19,12 +21,22 @@
 
 using namespace cpattn;
 
+// Streams and events of the host-buffer forward on one device, created at its first call and
+// kept until the plan is destroyed (e_in / e_comp: one pair per block of KV heads).
+struct HostPipe {
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t e_start = nullptr, e_done = nullptr;
+  std::vector<cudaEvent_t> e_in, e_comp;
+};
+
 struct cp_plan {
   cp_attn_config_t cfg;
   int G;
   float scale;
   mutable std::mutex mu;
   mutable std::map<int, int*> status_words;  // per device ordinal
+  mutable std::mutex host_mu;                // held while a host-buffer forward enqueues
+  mutable std::map<int, HostPipe> host_pipes;  // per device ordinal
 };
 
 namespace {
@@ -177,9 +189,14 @@ cp_status_t launch_permute(const void* in, void* out, int64_t B, int64_t X, int6
   p.in = static_cast<const uint4*>(in);
   p.out = static_cast<uint4*>(out);
   p.vec_per_row = static_cast<int>(row_bytes / 16);
+  p.vec_shift = -1;
+  for (int sh = 0; sh < 31; ++sh)
+    if ((1 << sh) == p.vec_per_row) p.vec_shift = sh;
+  // about kPermVecPerPass vectors per block: one pass of kPermVecPerThread loads per thread
+  p.rows_per_block = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kPermMaxRows, kPermVecPerPass / p.vec_per_row)));
   p.X = static_cast<int>(X);
   p.Y = static_cast<int>(Y);
-  p.n_vec = B * X * Y * p.vec_per_row;
+  p.n_rows = B * X * Y;
   const int64_t per = 16 / eb;
   p.in_sb = in_str[0] / per;
   p.in_sx = in_str[1] / per;
@@ -196,9 +213,8 @@ cp_status_t launch_permute(const void* in, void* out, int64_t B, int64_t X, int6
     if (n_ranks < 1 || L % (2 * n_ranks) != 0) return CP_ERR_INVALID_ARG;
     p.shard = static_cast<int>(L / (2 * n_ranks));
   }
-  if (p.n_vec == 0) return CP_OK;
-  const int64_t per_block = kPermThreads * kVecPerThread;
-  const int64_t grid = (p.n_vec + per_block - 1) / per_block;
+  if (p.n_rows == 0) return CP_OK;
+  const int64_t grid = (p.n_rows + p.rows_per_block - 1) / p.rows_per_block;
   permute_rows_kernel<<<(unsigned)grid, kPermThreads, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
@@ -377,6 +393,7 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
   }
   p.status = sw;
   p.wait_limit_ns = c.wait_limit_ns ? c.wait_limit_ns : kDefaultWaitLimitNs;
+  p.debug_fault = c.debug_fault;
   CUtensorMap mq, mk, mv, mdo;
   CP_TRY(make_map_bhld(&mq, vq.data, vq.B, vq.H, vq.L, vq.d, vq.sB, vq.sH, vq.sL));
   CP_TRY(make_map_bhld(&mk, vk.data, vk.B, vk.H, vk.L, vk.d, vk.sB, vk.sH, vk.sL));
@@ -421,6 +438,7 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
   }
   qp.status = sw;
   qp.wait_limit_ns = p.wait_limit_ns;
+  qp.debug_fault = c.debug_fault;
   const int64_t qgrid = (int64_t)qp.n_chunks * qp.tiles_per_chunk * c.B * c.Hq;
   if (c.d == 128) {
     CP_TRY(launch_bwd_dq_d<128>(qp, mq, mk, mv, mdo, qgrid, s));
@@ -483,7 +501,7 @@ cp_status_t cp_attn_plan(const cp_attn_config_t* cfg, cp_plan_t** out) {
       return CP_ERR_INVALID_ARG;
   }
   if (c.d != 64 && c.d != 128) return CP_ERR_UNSUPPORTED;
-  if (c.debug_fault < 0 || c.debug_fault > 1) return CP_ERR_INVALID_ARG;
+  if (c.debug_fault < 0 || c.debug_fault > 3) return CP_ERR_INVALID_ARG;
   cp_plan_t* p = new (std::nothrow) cp_plan_t();
   if (!p) return CP_ERR_INVALID_ARG;
   p->cfg = c;
@@ -499,6 +517,16 @@ void cp_attn_plan_destroy(cp_plan_t* plan) {
   cudaGetDevice(&prev);
   for (auto& kv : plan->status_words) {
     if (cudaSetDevice(kv.first) == cudaSuccess) cudaFree(kv.second);
+  }
+  for (auto& kv : plan->host_pipes) {
+    if (cudaSetDevice(kv.first) != cudaSuccess) continue;
+    HostPipe& hp = kv.second;
+    for (cudaEvent_t e : hp.e_in) cudaEventDestroy(e);
+    for (cudaEvent_t e : hp.e_comp) cudaEventDestroy(e);
+    if (hp.e_start) cudaEventDestroy(hp.e_start);
+    if (hp.e_done) cudaEventDestroy(hp.e_done);
+    if (hp.s_in) cudaStreamDestroy(hp.s_in);
+    if (hp.s_out) cudaStreamDestroy(hp.s_out);
   }
   if (prev >= 0) cudaSetDevice(prev);
   delete plan;
@@ -642,28 +670,42 @@ cp_status_t cp_attn_fwd_host(const cp_plan_t* plan, const cp_tensor_t* q, const 
   const size_t l_blk = (size_t)hb * G * c.L * 4;
   const int n_parts = c.B * nb;
 
-  cudaStream_t s_in = nullptr, s_out = nullptr;
-  cudaEvent_t e_start = nullptr, e_done = nullptr;
   cp_status_t st = CP_OK;
   auto cuda_ok = [&](cudaError_t e) {
     if (e != cudaSuccess && st == CP_OK) st = CP_ERR_CUDA;
     return st == CP_OK;
   };
-  if (!cuda_ok(cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking)) ||
-      !cuda_ok(cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking)) ||
-      !cuda_ok(cudaEventCreateWithFlags(&e_start, cudaEventDisableTiming)) ||
-      !cuda_ok(cudaEventCreateWithFlags(&e_done, cudaEventDisableTiming)) || !cuda_ok(cudaEventRecord(e_start, s)) ||
-      !cuda_ok(cudaStreamWaitEvent(s_in, e_start, 0)) || !cuda_ok(cudaStreamWaitEvent(s_out, e_start, 0))) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CP_ERR_CUDA;
+  // The plan's streams and events for this device (created at the first call).  The lock is
+  // held while this call enqueues: a wait captures an event's latest record when it is
+  // enqueued, so concurrent calls may reuse the events, one after the other.
+  std::lock_guard<std::mutex> guard(plan->host_mu);
+  HostPipe& hp = plan->host_pipes[dev];
+  if (!hp.s_in && !cuda_ok(cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking))) return st;
+  if (!hp.s_out && !cuda_ok(cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking))) return st;
+  if (!hp.e_start && !cuda_ok(cudaEventCreateWithFlags(&hp.e_start, cudaEventDisableTiming))) return st;
+  if (!hp.e_done && !cuda_ok(cudaEventCreateWithFlags(&hp.e_done, cudaEventDisableTiming))) return st;
+  while ((int)hp.e_in.size() < n_parts) {
+    cudaEvent_t a = nullptr, b2 = nullptr;
+    if (!cuda_ok(cudaEventCreateWithFlags(&a, cudaEventDisableTiming))) return st;
+    if (!cuda_ok(cudaEventCreateWithFlags(&b2, cudaEventDisableTiming))) {
+      cudaEventDestroy(a);
+      return st;
+    }
+    hp.e_in.push_back(a);
+    hp.e_comp.push_back(b2);
+  }
+  const cudaStream_t s_in = hp.s_in, s_out = hp.s_out;
+  if (!cuda_ok(cudaEventRecord(hp.e_start, s)) || !cuda_ok(cudaStreamWaitEvent(s_in, hp.e_start, 0)) ||
+      !cuda_ok(cudaStreamWaitEvent(s_out, hp.e_start, 0))) {
   } else {
     for (int part = 0; part < n_parts && st == CP_OK; ++part) {
       const int b = part / nb, kb = part - b * nb;
       const size_t qoff = ((size_t)b * c.Hq + (size_t)kb * hb * G) * c.L * c.d * 2;
       const size_t kvoff = ((size_t)b * c.Hkv + (size_t)kb * hb) * c.L * c.d * 2;
       const size_t loff = ((size_t)b * c.Hq + (size_t)kb * hb * G) * c.L * 4;
-      cudaEvent_t e_in = nullptr, e_comp = nullptr;
-      if (!cuda_ok(cudaEventCreateWithFlags(&e_in, cudaEventDisableTiming)) ||
-          !cuda_ok(cudaEventCreateWithFlags(&e_comp, cudaEventDisableTiming)))
-        break;
+      const cudaEvent_t e_in = hp.e_in[part], e_comp = hp.e_comp[part];
       // 1) this block's inputs in (behind the previous block's, on s_in)
       cuda_ok(cudaMemcpyAsync(dq + qoff, static_cast<const uint8_t*>(q->data) + qoff, q_blk, cudaMemcpyHostToDevice, s_in));
       cuda_ok(cudaMemcpyAsync(dk + kvoff, static_cast<const uint8_t*>(k->data) + kvoff, kv_blk, cudaMemcpyHostToDevice, s_in));
@@ -693,17 +735,11 @@ cp_status_t cp_attn_fwd_host(const cp_plan_t* plan, const cp_tensor_t* q, const 
       cuda_ok(cudaMemcpyAsync(static_cast<uint8_t*>(o->data) + qoff, dO + qoff, q_blk, cudaMemcpyDeviceToHost, s_out));
       cuda_ok(cudaMemcpyAsync(static_cast<uint8_t*>(lse->data) + loff, reinterpret_cast<uint8_t*>(dl) + loff, l_blk,
                               cudaMemcpyDeviceToHost, s_out));
-      cudaEventDestroy(e_in);   // released once recorded work completes
-      cudaEventDestroy(e_comp);
     }
     // the caller's stream continues only after the last block's outputs have landed
-    cuda_ok(cudaEventRecord(e_done, s_out));
-    cuda_ok(cudaStreamWaitEvent(s, e_done, 0));
+    cuda_ok(cudaEventRecord(hp.e_done, s_out));
+    cuda_ok(cudaStreamWaitEvent(s, hp.e_done, 0));
   }
-  if (e_start) cudaEventDestroy(e_start);
-  if (e_done) cudaEventDestroy(e_done);
-  if (s_in) cudaStreamDestroy(s_in);    // resources freed after the enqueued work completes
-  if (s_out) cudaStreamDestroy(s_out);
   return st;
 }
 
@@ -797,9 +833,10 @@ cp_status_t cp_lse_merge(cp_tensor_t* o_acc, cp_tensor_t* lse_acc, const cp_tens
                 lse_acc->stride[0], lse_acc->stride[1], lse_acc->stride[2],
                 o_part->stride[0], o_part->stride[1], o_part->stride[2],
                 lse_part->stride[0], lse_part->stride[1], lse_part->stride[2]};
-  const int64_t threads = B * H * R * (d / 4);
-  if (threads == 0) return CP_OK;
-  lse_merge_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, as_stream(stream)>>>(p);
+  if (B * H * R == 0) return CP_OK;
+  const int64_t rows_per_block = (32 / (d / 4)) * kMergeSlots * (kMergeThreads / 32);
+  const dim3 grid((unsigned)((R + rows_per_block - 1) / rows_per_block), (unsigned)std::min<int64_t>(B * H, 65535));
+  lse_merge_kernel<<<grid, kMergeThreads, 0, as_stream(stream)>>>(p);
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 

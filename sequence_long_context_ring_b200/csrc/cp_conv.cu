@@ -110,6 +110,7 @@ cp_status_t run_conv(const cp_conv_plan_t* plan, const cp_tensor_t* x, const cp_
     p.h_sd = h->stride[0];
     p.status = status;
     p.wait_limit_ns = c.wait_limit_ns ? c.wait_limit_ns : kConvDefaultWaitLimitNs;
+    p.debug_fault = c.debug_fault;
     const int sms = sm_count();
     if (sms <= 0) return CP_ERR_CUDA;
     const long long grid = p.n_tiles < sms ? p.n_tiles : sms;
@@ -164,6 +165,7 @@ cp_status_t cp_conv_plan(const cp_conv_config_t* cfg, cp_conv_plan_t** out) {
   if (c.lh < 1 || c.lh > kConvMaxTaps) return CP_ERR_INVALID_ARG;
   if (c.L % c.n_cp != 0) return CP_ERR_INVALID_ARG;
   if (c.lh - 1 > c.L / c.n_cp) return CP_ERR_INVALID_ARG;
+  if (c.debug_fault < 0 || c.debug_fault > 1) return CP_ERR_INVALID_ARG;
   if (static_cast<int64_t>(c.B) * c.D > 0x7fffffffLL) return CP_ERR_INVALID_ARG;
   cp_conv_plan_t* p = new (std::nothrow) cp_conv_plan_t();
   if (!p) return CP_ERR_INVALID_ARG;

@@ -55,6 +55,8 @@ def test_version_and_status_strings():
     (dict(split="zigzag", L=1028, n_cp=4), binding.CP_ERR_INVALID_ARG),   # two shards per rank: 2N | L
     (dict(split="striped", mode="ulysses", L=1020, n_cp=4), binding.CP_ERR_INVALID_ARG),
     (dict(B=0), binding.CP_ERR_INVALID_ARG),
+    (dict(debug_fault=4), binding.CP_ERR_INVALID_ARG),          # the fault seams are 1..3
+    (dict(debug_fault=-1), binding.CP_ERR_INVALID_ARG),
 ])
 def test_plan_validation_errors(kw, err):
     args = dict(B=1, Hq=8, Hkv=8, L=1024, d=128, n_cp=4)
@@ -122,6 +124,7 @@ def test_workspace_sizes():
     dict(L=1000, n_cp=3),                      # L % n_cp != 0
     dict(L=64, n_cp=4, lh=18),                 # halo of 17 > shard of 16
     dict(B=0), dict(D=0), dict(n_cp=0),
+    dict(debug_fault=2),                       # the one fault seam is 1
 ])
 def test_conv_plan_validation_errors(kw):
     args = dict(B=1, D=4, L=1024, lh=7, n_cp=4)
