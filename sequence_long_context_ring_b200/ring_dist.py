@@ -19,7 +19,9 @@ keys are full when b < a, masked (key <= query) when b == a, and skipped when b 
 step carries the same causal work under zig-zag, which is why the split is used.
 
 The exchange lands every remote shard in this rank's own memory before a kernel reads it;
-no kernel reads a peer's memory.
+no kernel reads a peer's memory.  It is injectable: the default passes the device buffers
+point to point over the group (NCCL); `host_staged_exchange` passes them through host memory,
+for process groups that move only host tensors (gloo), e.g. several ranks sharing one GPU.
 """
 from __future__ import annotations
 
@@ -57,6 +59,37 @@ def cuda_partial(q, k, v, diagonal: bool, scale: float):
     return _plans.get(B, Hq, k.shape[1], c, d, diagonal, scale).ring_step(0, 0, q, k, v)
 
 
+def p2p_exchange(send, recv, nxt: int, prv: int, group=None):
+    """Start sending `send` to rank `nxt` and receiving `recv` from rank `prv`; returns the
+    requests to wait on (after which `recv` holds the message)."""
+    return dist.batch_isend_irecv([dist.P2POp(dist.isend, send, nxt, group),
+                                   dist.P2POp(dist.irecv, recv, prv, group)])
+
+
+class _HostRecv:
+    """Completes a host-staged exchange: waits for the messages, then copies the received
+    host buffer into the device buffer (stream-ordered before any later kernel)."""
+
+    def __init__(self, reqs, host_recv, recv):
+        self.reqs, self.host_recv, self.recv = reqs, host_recv, recv
+
+    def wait(self):
+        for r in self.reqs:
+            r.wait()
+        self.recv.copy_(self.host_recv, non_blocking=False)
+
+
+def host_staged_exchange(send, recv, nxt: int, prv: int, group=None):
+    """The same exchange as p2p_exchange with the message staged through host memory: `send`
+    is copied to the host, sent over the group, and the received host message copied into
+    `recv` on wait().  For process groups whose backend moves only host tensors (gloo)."""
+    host_send = send.to("cpu")
+    host_recv = torch.empty_like(host_send)
+    reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, host_send, nxt, group),
+                                   dist.P2POp(dist.irecv, host_recv, prv, group)])
+    return [_HostRecv(reqs, host_recv, recv)]
+
+
 def shards_of_rank(split: str, n: int, r: int):
     """The two shard indices (of 2n) held by rank r under a two-shard split."""
     if split == "zigzag":
@@ -67,16 +100,20 @@ def shards_of_rank(split: str, n: int, r: int):
 
 
 def ring_attention(q, k, v, group=None, *, causal: bool = True, scale: float = 0.0, split: str = "contiguous",
-                   partial_fn: Optional[Callable] = None, merge_fn: Optional[Callable] = None):
+                   partial_fn: Optional[Callable] = None, merge_fn: Optional[Callable] = None,
+                   exchange_fn: Optional[Callable] = None):
     """This rank's share of ring attention over the process group.
 
     q [B, Hq, c, d], k, v [B, Hkv, c, d]: this rank's rows (contiguous: sequence positions
     [r c, (r+1) c); zigzag / striped: its two shards of c/2 positions, in order).  Returns
     (O [B, Hq, c, d] normalised, LSE [B, Hq, c]) of this rank's queries over the whole
     sequence, in fp32 on the GPU.  partial_fn(q, k, v, diagonal, scale) -> (O, LSE) and
-    merge_fn(acc_o, acc_lse, o, lse) (in place) default to the library's kernels."""
+    merge_fn(acc_o, acc_lse, o, lse) (in place) default to the library's kernels;
+    exchange_fn(send, recv, next_rank, prev_rank, group) -> waitables defaults to
+    p2p_exchange."""
     partial_fn = partial_fn or cuda_partial
     merge_fn = merge_fn or lse_merge
+    exchange_fn = exchange_fn or p2p_exchange
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     nxt, prv = (rank + 1) % world, (rank - 1) % world
@@ -94,8 +131,7 @@ def ring_attention(q, k, v, group=None, *, causal: bool = True, scale: float = 0
         reqs = []
         if s < world - 1:
             # pass the shard held now to the next rank, receive the next one from the previous
-            reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, kv_cur, nxt, group),
-                                           dist.P2POp(dist.irecv, kv_nxt, prv, group)])
+            reqs = exchange_fn(kv_cur, kv_nxt, nxt, prv, group)
         if split == "contiguous":
             if not (causal and j > rank):
                 po, pl = partial_fn(q, kv_cur[0], kv_cur[1], causal and j == rank, scale)

@@ -33,7 +33,7 @@ def _positions(split, world, L, r):
     return osp.rank_positions(split, world, L, r)
 
 
-def _rank(rank, world, port, causal, split, out):
+def _rank(rank, world, port, causal, split, out, staged=False):
     import torch
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
@@ -68,7 +68,9 @@ def _rank(rank, world, port, causal, split, out):
             acc_o.copy_(torch.from_numpy(o2))
             acc_l.copy_(torch.from_numpy(l2))
 
-        o, lse = ring_dist.ring_attention(qr, kr, vr, causal=causal, split=split, partial_fn=partial, merge_fn=merge)
+        exchange = ring_dist.host_staged_exchange if staged else None
+        o, lse = ring_dist.ring_attention(qr, kr, vr, causal=causal, split=split, partial_fn=partial, merge_fn=merge,
+                                          exchange_fn=exchange)
         out[rank] = (o.numpy(), lse.numpy(), calls)
     finally:
         dist.destroy_process_group()
@@ -108,6 +110,24 @@ def test_ring_across_processes_equals_full_attention(world, causal, split):
             assert len(calls) == n_pairs and sum(calls) == 2
             if split == "zigzag":
                 assert n_pairs == 3 + 2 * (world - 1)
+
+
+@pytest.mark.parametrize("world,split", [(3, "zigzag"), (4, "contiguous")])
+def test_host_staged_exchange_gives_the_same_ring(world, split):
+    # the exchange through host buffers (for groups that move only host tensors) runs the same
+    # schedule: every rank's rows equal full attention
+    import oracle
+    port = 29550 + (os.getpid() * 5 + world * 17 + len(split)) % 2000
+    with mp.get_context("spawn").Manager() as man:
+        out = man.dict()
+        mp.spawn(_rank, args=(world, port, True, split, out, True), nprocs=world, join=True)
+        res = dict(out)
+    q, k, v = _inputs(world)
+    o_ref, l_ref = oracle.attention_full(q, k, v)
+    for r in range(world):
+        pos = _positions(split, world, q.shape[2], r)
+        np.testing.assert_allclose(res[r][0], o_ref[:, :, pos], atol=1e-12)
+        np.testing.assert_allclose(res[r][1], l_ref[:, :, pos], atol=1e-12)
 
 
 def ring_dist_shards(split, world, r):
