@@ -7,25 +7,42 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
+from oracle import split as osp
+from sequence_long_context_ring_b200 import synth
 from sequence_long_context_ring_b200.binding import Plan, CpError, CP_ERR_WORKSPACE, CP_ERR_INVALID_ARG
 
 from _helpers import to_dev, to_f64, inputs, assert_attn_close
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("mode,n_cp,n_hp", [("ulysses", 4, 1), ("2d", 2, 2)])
-def test_noalloc_matches_workspace_entry_point_twice(cuda_lib, mode, n_cp, n_hp):
+@pytest.mark.parametrize("mode,n_cp,n_hp,split", [("ulysses", 4, 1, "contiguous"), ("2d", 2, 2, "contiguous"),
+                                                  ("ulysses", 4, 1, "zigzag")])
+def test_noalloc_matches_workspace_entry_point_twice(cuda_lib, mode, n_cp, n_hp, split):
+    # Both entry points run the same kernels on the same inputs, so their results must agree
+    # bit for bit; the first is also checked against the fp64 oracle.  Two calls in a row with
+    # different inputs: nothing left in the shared scratch by the first may leak into the second.
     B, L, Hq, Hkv, d = 1, 1024, 8, 4, 128
-    plan = Plan(B, Hq, Hkv, L, d, n_cp=n_cp, n_hp=n_hp, mode=mode)
+    plan = Plan(B, Hq, Hkv, L, d, n_cp=n_cp, n_hp=n_hp, mode=mode, split=split)
     assert plan.workspace_size() <= 64 << 20
-    for call, seed in enumerate((71, 72)):   # two calls in a row, different inputs
-        q, k, v = (to_dev(x) for x in inputs(seed, (B, L, Hq, d), (B, L, Hkv, d)))
-        o_ref, lse_ref = plan.fwd(q, k, v)
-        o = torch.full_like(o_ref, float("nan"))
-        lse = torch.full_like(lse_ref, float("nan"))
+    for call, seed in enumerate((71, 72)):
+        qb, kb, vb = inputs(seed, (B, L, Hq, d), (B, L, Hkv, d))
+        q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+        o_ws, lse_ws = plan.fwd(q, k, v)
+        o = torch.full_like(o_ws, float("nan"))
+        lse = torch.full_like(lse_ws, float("nan"))
         plan.fwd_noalloc(q, k, v, o, lse)
         torch.cuda.synchronize()
-        assert_attn_close(to_f64(o), to_f64(o_ref), to_f64(lse), to_f64(lse_ref), f"{mode} call {call}")
+        assert torch.equal(o.view(torch.int16), o_ws.view(torch.int16)), f"{mode}/{split} call {call}: O differs"
+        assert torch.equal(lse, lse_ws), f"{mode}/{split} call {call}: LSE differs"
+        q64, k64, v64 = (synth.bf16_bits_to_f64(x) for x in (qb, kb, vb))
+        if mode == "2d":
+            o_ref, l_ref = oracle.attention_2d(q64, k64, v64, n_hp, n_cp)
+        elif split == "contiguous":
+            o_ref, l_ref = oracle.ulysses_attention(q64, k64, v64, n_cp)
+        else:
+            o_ref, l_ref = osp.ulysses_attention_split(q64, k64, v64, n_cp, split)
+        assert_attn_close(to_f64(o), o_ref, to_f64(lse), l_ref, f"{mode}/{split} call {call} vs oracle")
 
 
 @pytest.mark.gpu
