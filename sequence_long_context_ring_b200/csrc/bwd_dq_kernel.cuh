@@ -253,32 +253,36 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_kk = make_idesc_bf16(128, 128, false);  // S, dP: A and B K-major
       constexpr uint32_t idesc_o = make_idesc_bf16(128, D, true);      // dQ: A TMEM, B (K) N-major
-      const uint32_t q_a = smem_u32(q_s), do_a = smem_u32(do_s), k_a0 = smem_u32(k_s), v_a0 = smem_u32(v_s);
+      // Operand descriptors, built once: Q, dO, and slot 0 of K and V as K-major tiles, slot 0 of K
+      // as the N-major B of dQ; a slot's descriptor is slot 0's plus the slot offset.
+      const uint32_t q_d = sdesc_lo(smem_u32(q_s), 16), do_d = sdesc_lo(smem_u32(do_s), 16);
+      const uint32_t k_d0 = sdesc_lo(smem_u32(k_s), 16), v_d0 = sdesc_lo(smem_u32(v_s), 16);
+      const uint32_t kn_d0 = sdesc_lo(smem_u32(k_s), kBoxBytes);
       // X = A B^T over d (both tiles d-contiguous), 128 x 128 into TMEM column d_tmem
       auto issue_kk = [=](uint32_t d_tmem, uint32_t a, uint32_t b) {
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          umma_ss(d_tmem, make_sdesc(a + off, 16, 1024), make_sdesc(b + off, 16, 1024), idesc_kk, kk > 0 ? 1u : 0u);
+          umma_ss(d_tmem, sdesc_lo_at(a, off), sdesc_lo_at(b, off), idesc_kk, kk > 0 ? 1u : 0u);
         }
       };
       auto wait_k = [&](int i) { return wait_bounded(&k_full[i % kDqKSlots], (i / kDqKSlots) & 1, ctl, kQSiteMmaK); };
       auto wait_v = [&](int i) {
         return wait_bounded(&v_full[i % kDqVSlots], (i / kDqVSlots) & 1, ctl, kQSiteMmaV);
       };
-      auto kaddr = [&](int i) { return k_a0 + (i % kDqKSlots) * kTile; };
-      auto vaddr = [&](int i) { return v_a0 + (i % kDqVSlots) * kTile; };
+      auto kdesc = [&](int i) { return sdesc_lo_at(k_d0, (i % kDqKSlots) * kTile); };
+      auto vdesc = [&](int i) { return sdesc_lo_at(v_d0, (i % kDqVSlots) * kTile); };
 
       bool ok = wait_bounded(q_full, 0, ctl, kQSiteMmaQ);
       if (ok && T > 0) {
         ok = wait_k(0);
         if (ok) {
-          issue_kk(tS0, q_a, kaddr(0));
+          issue_kk(tS0, q_d, kdesc(0));
           umma_commit(&s_full[0]);
           ok = wait_v(0);
         }
         if (ok) {
-          issue_kk(tDP, do_a, vaddr(0));
+          issue_kk(tDP, do_d, vdesc(0));
           umma_commit(&dp_full[0]);
         }
       }
@@ -286,23 +290,23 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         if (i + 1 < T) {
           // S(i+1) into buffer (i+1)&1, which held dS(i-1): dQ(i-1) was issued before
           if (!wait_k(i + 1)) { ok = false; break; }
-          issue_kk(tS0 + ((i + 1) & 1) * 128, q_a, kaddr(i + 1));
+          issue_kk(tS0 + ((i + 1) & 1) * 128, q_d, kdesc(i + 1));
           umma_commit(&s_full[(i + 1) & 1]);
           // dP(i+1) over dP(i), once the elementwise warps hold dP(i) in registers
           if (!wait_v(i + 1)) { ok = false; break; }
           if (!wait_bounded(dp_free, i & 1, ctl, kQSiteMmaDpFree)) { ok = false; break; }
           tc_fence_after();
-          issue_kk(tDP, do_a, vaddr(i + 1));
+          issue_kk(tDP, do_d, vdesc(i + 1));
           umma_commit(&dp_full[(i + 1) & 1]);
         }
         // dQ += dS(i) K(i): A = dS from TMEM (8 columns per 16 keys), B = K N-major
         if (!wait_bounded(&ds_full[i & 1], (i >> 1) & 1, ctl, kQSiteMmaDs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ds_t = tS0 + (i & 1) * 128;
-        const uint32_t ka = kaddr(i);
-#pragma unroll 1
+        const uint32_t kn = sdesc_lo_at(kn_d0, (i % kDqKSlots) * kTile);
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // keys [16 kk, 16 kk + 16): written by warpgroup kk / 4
-          umma_ts(tDQ, ds_t + 64u * (kk >> 2) + 8u * (kk & 3), make_sdesc(ka + kk * 2048, kBoxBytes, 1024), idesc_o,
+          umma_ts(tDQ, ds_t + 64u * (kk >> 2) + 8u * (kk & 3), sdesc_lo_at(kn, kk * 2048), idesc_o,
                   (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&k_free[i % kDqKSlots]);
       }

@@ -277,15 +277,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_kk = make_idesc_bf16(128, 128, false);     // S^T, dP^T: both K-major
       constexpr uint32_t idesc_tn = make_idesc_bf16(128, D, true);        // dV, dK: A TMEM, B N-major
-      const uint32_t k_a = smem_u32(k_s), v_a = smem_u32(v_s);
-      auto q_addr = [&](int i) { return smem_u32(q_s + (i & 1) * kTile); };
-      auto do_addr = [&](int i) { return smem_u32(do_s + (i & 1) * kTile); };
+      // Operand descriptors, built once: K and V as K-major A tiles; stage 0 of Q and dO both as
+      // K-major B tiles (S^T, dP^T) and as N-major B tiles (dK, dV); stage 1 is one tile later.
+      const uint32_t k_d = sdesc_lo(smem_u32(k_s), 16), v_d = sdesc_lo(smem_u32(v_s), 16);
+      const uint32_t q_k0 = sdesc_lo(smem_u32(q_s), 16), do_k0 = sdesc_lo(smem_u32(do_s), 16);
+      const uint32_t q_n0 = sdesc_lo(smem_u32(q_s), kBoxBytes), do_n0 = sdesc_lo(smem_u32(do_s), kBoxBytes);
+      auto stage = [&](uint32_t d0, int i) { return sdesc_lo_at(d0, (i & 1) * kTile); };
       // S^T(i) = K Q_i^T and dP^T(i) = V dO_i^T  [M = keys, N = queries, K = d]
       auto issue_kk = [&](uint32_t d_tmem, uint32_t a, uint32_t b) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          umma_ss(d_tmem, make_sdesc(a + off, 16, 1024), make_sdesc(b + off, 16, 1024), idesc_kk, kk > 0);
+          umma_ss(d_tmem, sdesc_lo_at(a, off), sdesc_lo_at(b, off), idesc_kk, kk > 0);
         }
       };
       bool ok = wait_bounded(kv_full, 0, ctl, kBSiteMmaKV);
@@ -293,9 +296,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = wait_bounded(&q_full[0], 0, ctl, kBSiteMmaQ);
         if (ok) {
           tc_fence_after();
-          issue_kk(tS, k_a, q_addr(0));
+          issue_kk(tS, k_d, stage(q_k0, 0));
           umma_commit(s_full);
-          issue_kk(tDP, v_a, do_addr(0));
+          issue_kk(tDP, v_d, stage(do_k0, 0));
           umma_commit(dp_full);
         }
       }
@@ -304,29 +307,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // (1) dV += P^T dO  [A = P^T in TMEM (keys x queries), B = dO N-major]
         if (!wait_bounded(p_full, i & 1, ctl, kBSiteMmaP)) { ok = false; break; }
         tc_fence_after();
+        {
+          const uint32_t b = stage(do_n0, i);
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tDV, tS + bwd_a_col(kk), make_sdesc(do_addr(i) + kk * 2048, kBoxBytes, 1024), idesc_tn,
-                  (i > 0 || kk > 0));
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            umma_ts(tDV, tS + bwd_a_col(kk), sdesc_lo_at(b, kk * 2048), idesc_tn, (i > 0 || kk > 0));
+        }
         // (2) S^T(i+1) over P^T(i) (read by dV(i), issued before)
         const bool more = i + 1 < it.n_iter;
         if (more) {
           if (!wait_bounded(&q_full[st ^ 1], ((i + 1) >> 1) & 1, ctl, kBSiteMmaQ)) { ok = false; break; }
           tc_fence_after();
-          issue_kk(tS, k_a, q_addr(i + 1));
+          issue_kk(tS, k_d, stage(q_k0, i + 1));
           umma_commit(s_full);
         }
         // (3) dK += dS^T Q  [A = dS^T in TMEM, B = Q N-major]; then stage i is free
         if (!wait_bounded(ds_full, i & 1, ctl, kBSiteMmaDs)) { ok = false; break; }
         tc_fence_after();
+        {
+          const uint32_t b = stage(q_n0, i);
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tDK, tDP + bwd_a_col(kk), make_sdesc(q_addr(i) + kk * 2048, kBoxBytes, 1024), idesc_tn,
-                  (i > 0 || kk > 0));
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            umma_ts(tDK, tDP + bwd_a_col(kk), sdesc_lo_at(b, kk * 2048), idesc_tn, (i > 0 || kk > 0));
+        }
         umma_commit(&q_empty[st]);
         // (4) dP^T(i+1) over dS^T(i) (read by dK(i), issued before)
         if (more) {
-          issue_kk(tDP, v_a, do_addr(i + 1));
+          issue_kk(tDP, v_d, stage(do_k0, i + 1));
           umma_commit(dp_full);
         }
       }

@@ -235,6 +235,11 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc_bf16(128, 128, false);
       const int kk_prev = p.lh > 1 ? p.kk1 : 8;       // K steps of the previous block with taps
+      // descriptors built once: stage 0's current-block and previous-block views (the latter
+      // one 128-byte row earlier) and the two Toeplitz tiles
+      const uint32_t cur0 = smem0 + S::kStage0 + kConvLead * 128;                     // atom-aligned
+      const uint32_t cur_d0 = sdesc_lo(cur0, 16), prev_d0 = sdesc_lo(cur0 - 128, 16);
+      const uint32_t t0_d = sdesc_lo(smem0 + S::kT0, 16), t1_d = sdesc_lo(smem0 + S::kT1, 16);
       int rebuilds = 0, last_row = -1;
       bool ok = true;
       for (int i = 0; i < n_local && ok; ++i) {
@@ -250,19 +255,18 @@ __global__ void __launch_bounds__(kConvThreads, 1)
         if (i >= 2 && !wait_bounded(&tempty[a], ((i >> 1) - 1) & 1, ctl, kCSiteMmaAcc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem_base + a * 128;
-        const uint32_t cur = smem0 + S::kStage0 + s * S::kStageBytes + kConvLead * 128;   // atom-aligned
-        const uint32_t prev = cur - 128;                                                   // one row earlier
+        const uint32_t cur_d = sdesc_lo_at(cur_d0, s * S::kStageBytes);
+        const uint32_t prev_d = sdesc_lo_at(prev_d0, s * S::kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kConvInBox + (kk & 3) * 32;
           const uint32_t toff = (kk >> 2) * kConvBox + (kk & 3) * 32;
-          umma_ss(d, make_sdesc(cur + off, 16, 1024), make_sdesc(smem0 + S::kT0 + toff, 16, 1024), idesc,
-                  kk > 0 ? 1u : 0u);
+          umma_ss(d, sdesc_lo_at(cur_d, off), sdesc_lo_at(t0_d, toff), idesc, kk > 0 ? 1u : 0u);
         }
         for (int kk = kk_prev; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kConvInBox + (kk & 3) * 32;
           const uint32_t toff = (kk >> 2) * kConvBox + (kk & 3) * 32;
-          umma_ss(d, make_sdesc(prev + off, 16, 1024), make_sdesc(smem0 + S::kT1 + toff, 16, 1024), idesc, 1u);
+          umma_ss(d, sdesc_lo_at(prev_d, off), sdesc_lo_at(t1_d, toff), idesc, 1u);
         }
         umma_commit(&empty[s]);
         umma_commit(&tfull[a]);

@@ -346,31 +346,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc_bf16(128, kBN, false);
       constexpr uint32_t idesc_o = make_idesc_bf16(128, D, true);
-      const uint32_t q_addr0 = smem_u32(q_smem);
-      const uint32_t kv_addr0 = smem_u32(kv_smem);
+      // Operand descriptors, built once: the two Q tiles and ring slot 0 as K-major tiles, ring
+      // slot 0 as an N-major tile (V); a slot's descriptor is slot 0's plus the slot offset.
+      const uint32_t q_d0 = sdesc_lo(smem_u32(q_smem), 16);
+      const uint32_t kv_k0 = sdesc_lo(smem_u32(kv_smem), 16);
+      const uint32_t kv_n0 = sdesc_lo(smem_u32(kv_smem), kBoxBytes);
 
       // S_ab = Q_ab K^T: M=128, N=128, K=D in steps of 16 (32 bytes inside a 128-byte swizzled row)
       auto issue_s = [=](int ab, int st) {
-        const uint32_t kaddr = kv_addr0 + st * kTileBytes;
-        const uint32_t qaddr = q_addr0 + ab * kTileBytes;
+        const uint32_t kd = sdesc_lo_at(kv_k0, st * kTileBytes);
+        const uint32_t qd = sdesc_lo_at(q_d0, ab * kTileBytes);
         const uint32_t d_tmem = tmem_base + ab * 256;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          umma_ss(d_tmem, make_sdesc(qaddr + off, 16, 1024), make_sdesc(kaddr + off, 16, 1024), idesc_s,
-                  kk > 0 ? 1u : 0u);
+          umma_ss(d_tmem, sdesc_lo_at(qd, off), sdesc_lo_at(kd, off), idesc_s, kk > 0 ? 1u : 0u);
         }
       };
       // O_ab += P_ab V over keys [64 h, 64 h + 64): A = P from TMEM (8 columns per 16 keys),
       // B = V N-major (d contiguous)
       auto issue_pv = [=](int ab, int st, int h, bool acc) {
-        const uint32_t vaddr = kv_addr0 + st * kTileBytes;
+        const uint32_t vd = sdesc_lo_at(kv_n0, st * kTileBytes);
         const uint32_t p_tmem = tmem_base + ab * 256;
         const uint32_t o_tmem = tmem_base + 128 + ab * 256;
 #pragma unroll
         for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
-          umma_ts(o_tmem, p_tmem + kk * 8, make_sdesc(vaddr + kk * 2048, kBoxBytes, 1024), idesc_o,
-                  (acc || kk > 0) ? 1u : 0u);
+          umma_ts(o_tmem, p_tmem + kk * 8, sdesc_lo_at(vd, kk * 2048), idesc_o, (acc || kk > 0) ? 1u : 0u);
         }
       };
       // both halves of PV_ab, each after its half of P is in TMEM

@@ -128,17 +128,30 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // ---- tcgen05: UMMA ---------------------------------------------------------------------------
-// Shared-memory matrix descriptor (sm_100 format): start address >> 4 in bits 0..13, leading
-// byte offset >> 4 in bits 16..29, stride byte offset >> 4 in bits 32..45, version 1 in bits
-// 46..47, swizzle mode in bits 61..63 (2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= 1ull << 46;
-  d |= 2ull << 61;
-  return d;
+// Shared-memory matrix descriptor (sm_100 format, 64 bits): start address >> 4 in bits 0..13,
+// leading byte offset >> 4 in bits 16..29, stride byte offset >> 4 in bits 32..45, version 1
+// in bits 46..47, swizzle mode in bits 61..63 (2 = 128-byte swizzle).
+// Every operand tile here uses a stride byte offset of 1024, version 1 and the 128-byte
+// swizzle, so all descriptors share one high word; only the low word (start address, leading
+// byte offset) differs.  Issuers keep a tile's low word and step through its K slices with
+// compile-time byte offsets (sdesc_lo_at); the MMA wrappers below pair the low word with the
+// constant high word inside the instruction's asm.  Building both 64-bit descriptors for every
+// MMA put a chain of dependent integer operations in front of each tcgen05.mma of the one
+// issuing thread, which (measured on B200) made issue, not the tensor pipe, the limit: about
+// 110-210 cycles per M = 128, N = 128, K = 16 MMA, against 64 with descriptors built in advance.
+constexpr uint32_t kSdescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+// The low word of the same layout `byte_off` bytes later.  The start-address field holds
+// addr >> 4 in its low 14 bits and every shared-memory address fits there, so the add never
+// carries out of the field.  An ordered asm statement, so each word is formed right before its
+// MMA instead of a whole loop's words being hoisted into registers (the forward's MMA issuer
+// runs under a 72-register cap).
+__device__ __forceinline__ uint32_t sdesc_lo_at(uint32_t lo, uint32_t byte_off) {
+  uint32_t r;
+  asm volatile("add.u32 %0, %1, %2;" : "=r"(r) : "r"(lo), "r"(byte_off >> 4));
+  return r;
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
@@ -149,24 +162,29 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_mn_m
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A[smem] * B[smem], operands given by their descriptors' low words
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
                                         uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p;\n\t.reg .b32 hi;\n\t.reg .b64 da, db;\n\t"
+      "mov.b32 hi, %5;\n\t"
+      "mov.b64 da, {%1, hi};\n\t"
+      "mov.b64 db, {%2, hi};\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi)
       : "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem desc]
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A[tmem] * B[smem], B given by its descriptor's low word
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
                                         uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p;\n\t.reg .b32 hi;\n\t.reg .b64 db;\n\t"
+      "mov.b32 hi, %5;\n\t"
+      "mov.b64 db, {%2, hi};\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi)
       : "memory");
 }
 // Arrive once on `bar` when every tcgen05 MMA issued so far by this thread has completed.
