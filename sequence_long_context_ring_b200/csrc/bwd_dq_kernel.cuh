@@ -364,14 +364,20 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             if (cc * 32 + e >= lim) r[e] = __float_as_uint(-INFINITY);
         }
         uint32_t pk[16];
+        // every exponential of the chunk first, then dS = P (dP - D) and the bf16 packs
+        float pv[32];
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * e2]), __uint_as_float(r[2 * e2 + 1])), sl2x2, nl2), x0, x1);
-          const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          pv[2 * e2] = ex2_approx(x0);
+          pv[2 * e2 + 1] = ex2_approx(x1);
+        }
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
           const uint64_t dd = f2_add(f2_pack(__uint_as_float(g[2 * e2]), __uint_as_float(g[2 * e2 + 1])), nD2);
           float d0, d1;
-          f2_unpack(f2_mul(pp, dd), d0, d1);
+          f2_unpack(f2_mul(f2_pack(pv[2 * e2], pv[2 * e2 + 1]), dd), d0, d1);
           pk[e2] = pack_bf16x2(d0, d1);
         }
         tmem_st16(tS + cc * 16, pk);

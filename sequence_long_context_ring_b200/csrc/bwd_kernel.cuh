@@ -36,6 +36,7 @@
 namespace cpattn {
 
 constexpr int kBwdThreads = 320;
+
 constexpr int kBwdLoadWarp = 8;
 constexpr int kBwdMmaWarp = 9;
 
@@ -374,24 +375,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // P = 2^(S^T * scale * log2(e) - LSE * log2(e)) for one 32-column chunk, four columns
       // (two pairs) per -LSE vector
       auto p_chunk = [&](const uint32_t (&r)[32], int cc) {
+        // every exponential of the chunk first, then the masks and the bf16 packs
+        float pv[32];
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           const float4 nl = nls4[cc * 8 + e4];
-          const int e = 4 * e4, c = cc * 32 + e;
+          const int e = 4 * e4;
           float x0, x1, x2, x3;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), sl2x2, f2_pack(nl.x, nl.y)), x0,
                     x1);
           f2_unpack(f2_fma(f2_pack(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])), sl2x2, f2_pack(nl.z, nl.w)),
                     x2, x3);
-          float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+          pv[e] = ex2_approx(x0);
+          pv[e + 1] = ex2_approx(x1);
+          pv[e + 2] = ex2_approx(x2);
+          pv[e + 3] = ex2_approx(x3);
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int c = cc * 32 + e;
+          float p0 = pv[e], p1 = pv[e + 1];
           if (masked) {
             if (!kv_live || c < c_lo) p0 = 0.f;
             if (!kv_live || c + 1 < c_lo) p1 = 0.f;
-            if (!kv_live || c + 2 < c_lo) p2 = 0.f;
-            if (!kv_live || c + 3 < c_lo) p3 = 0.f;
           }
           pk[c >> 1] = pack_bf16x2(p0, p1);
-          pk[(c >> 1) + 1] = pack_bf16x2(p2, p3);
         }
       };
       p_chunk(ra, 0);

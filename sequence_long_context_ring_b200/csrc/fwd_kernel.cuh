@@ -451,34 +451,42 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       return fmax3(a, b, fmaxf(__uint_as_float(r[30]), __uint_as_float(r[31])));
     };
     // 2^(s*sl2 - m) of one 32-column chunk -> 16 packed bf16 columns of P written over S
-    // columns already read (P columns [16cc, 16cc+16)); returns the chunk's sum.  emu: a share
-    // of the pairs runs on the FMA pipe (only for chunks without masked columns, whose
-    // exponentials must be exact zeros).
+    // columns already read (P columns [16cc, 16cc+16)); returns the chunk's sum.  All the
+    // chunk's exponentials are issued before their results are summed (two chains) and packed:
+    // consuming each result at once stalled the warp on the MUFU latency.  emu: a share of the
+    // pairs runs on the FMA pipe (only for chunks without masked columns, whose exponentials
+    // must be exact zeros).
     auto exp_chunk = [&](const uint32_t (&r)[32], int cc, uint64_t negm2, bool emu) {
-      uint64_t sum2 = f2_pack(0.f, 0.f);
+      float pv[32];
+#pragma unroll
+      for (int e2 = 0; e2 < 16; ++e2) {
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * e2]), __uint_as_float(r[2 * e2 + 1])), sl2x2, negm2), x0,
+                  x1);
+        if (kEmuPairs > 0 && emu && (e2 * kEmuPairs) % 16 < kEmuPairs) {
+          ex2_fma2(x0, x1, pv[2 * e2], pv[2 * e2 + 1]);
+        } else {
+          pv[2 * e2] = ex2_approx(x0);
+          pv[2 * e2 + 1] = ex2_approx(x1);
+        }
+      }
+      uint64_t s0 = f2_pack(0.f, 0.f), s1 = s0;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int e2 = h * 8 + e;
-          float x0, x1, p0, p1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * e2]), __uint_as_float(r[2 * e2 + 1])), sl2x2, negm2), x0,
-                    x1);
-          if (kEmuPairs > 0 && emu && (e2 * kEmuPairs) % 16 < kEmuPairs) {
-            ex2_fma2(x0, x1, p0, p1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          sum2 = f2_add(sum2, f2_pack(p0, p1));
-          pk[e] = pack_bf16x2(p0, p1);
+          const uint64_t pp = f2_pack(pv[2 * e2], pv[2 * e2 + 1]);
+          if (e & 1) s1 = f2_add(s1, pp); else s0 = f2_add(s0, pp);
+          pk[e] = pack_bf16x2(pv[2 * e2], pv[2 * e2 + 1]);
         }
         tmem_st8(tS + cc * 16 + h * 8, pk);
       }
-      float a0, a1;
-      f2_unpack(sum2, a0, a1);
-      return a0 + a1;
+      float a0, a1, b0, b1;
+      f2_unpack(s0, a0, a1);
+      f2_unpack(s1, b0, b1);
+      return (a0 + a1) + (b0 + b1);
     };
     // all stores of this thread's P are in TMEM before one lane of the warp arrives
     auto publish = [&](uint64_t* bar) {
