@@ -1,7 +1,9 @@
 """The benchmark's reference arm on CPU: the timed fp64 oracle on a bounded sample prints the one
 JSON line of the contract (rank 0 only; any other rank exits 0 without work or output)."""
+import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 
@@ -66,3 +68,31 @@ def test_traffic_figure_is_dropped_once_the_kernel_changes(monkeypatch):
     assert bench.traffic_from_profile(w) == rec["per_launch_bytes"][w]
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
     assert bench.traffic_from_profile(w) is None
+
+
+def _csrc_hash(files):
+    """First 16 hex digits of sha256 over the kernel sources' bytes, in the order given."""
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "sequence_long_context_ring_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def test_every_profile_summary_matches_the_current_kernel_source():
+    """Each ncu summary under profiles/ names the kernel sources it was captured from, with a
+    hash of their bytes; once any of them changes, the summary is stale and must be captured
+    again (and this test fails until it is)."""
+    line = re.compile(r"^Source hash: ([0-9a-f]{16}) over (.+?)\s*$", re.M)
+    pdir = os.path.join(ROOT, "profiles")
+    names = sorted(f for f in os.listdir(pdir) if f.endswith(".md"))
+    assert names, "no ncu summaries"
+    for fn in names:
+        with open(os.path.join(pdir, fn)) as fh:
+            m = line.search(fh.read())
+        assert m, f"{fn}: no 'Source hash: <hex> over <files>' line"
+        files = [x.strip() for x in m.group(2).split(",")]
+        assert _csrc_hash(files) == m.group(1), f"{fn}: captured from kernel sources that have changed since"
+    with open(os.path.join(pdir, "ring_fwd_kernel_traffic.json")) as fh:
+        d = json.load(fh)
+    assert d["kernel_source_hash"] == _csrc_hash(["fwd_kernel.cuh", "sm100.cuh"]), "traffic figure is stale"
