@@ -356,9 +356,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dp_free);
-      // dS of one 32-key chunk -> 16 packed bf16 columns
-      auto ds_chunk = [&](uint32_t (&r)[32], const uint32_t (&g)[32], int cc) {
-        if (masked) {
+      // dS of one 32-key chunk -> 16 packed bf16 columns; the mask code exists only in the
+      // masked instance
+      auto ds_chunk = [&](uint32_t (&r)[32], const uint32_t (&g)[32], int cc, auto with_mask) {
+        if constexpr (decltype(with_mask)::value) {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             if (cc * 32 + e >= lim) r[e] = __float_as_uint(-INFINITY);
@@ -382,8 +383,13 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         tmem_st16(tS + cc * 16, pk);
       };
-      ds_chunk(sa, dpa, 0);
-      ds_chunk(sb, dpb, 1);
+      if (masked) {
+        ds_chunk(sa, dpa, 0, Flag<true>{});
+        ds_chunk(sb, dpb, 1, Flag<true>{});
+      } else {
+        ds_chunk(sa, dpa, 0, Flag<false>{});
+        ds_chunk(sb, dpb, 1, Flag<false>{});
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

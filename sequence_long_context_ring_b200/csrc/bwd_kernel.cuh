@@ -373,8 +373,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_wait_ld();
       uint32_t pk[32];  // P^T of the 64 columns as bf16 pairs, kept for dS
       // P = 2^(S^T * scale * log2(e) - LSE * log2(e)) for one 32-column chunk, four columns
-      // (two pairs) per -LSE vector
-      auto p_chunk = [&](const uint32_t (&r)[32], int cc) {
+      // (two pairs) per -LSE vector; the mask code exists only in the masked instance
+      auto p_chunk = [&](const uint32_t (&r)[32], int cc, auto with_mask) {
         // every exponential of the chunk first, then the masks and the bf16 packs
         float pv[32];
 #pragma unroll
@@ -395,15 +395,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int e = 0; e < 32; e += 2) {
           const int c = cc * 32 + e;
           float p0 = pv[e], p1 = pv[e + 1];
-          if (masked) {
+          if constexpr (decltype(with_mask)::value) {
             if (!kv_live || c < c_lo) p0 = 0.f;
             if (!kv_live || c + 1 < c_lo) p1 = 0.f;
           }
           pk[c >> 1] = pack_bf16x2(p0, p1);
         }
       };
-      p_chunk(ra, 0);
-      p_chunk(rb, 1);
+      if (masked) {
+        p_chunk(ra, 0, Flag<true>{});
+        p_chunk(rb, 1, Flag<true>{});
+      } else {
+        p_chunk(ra, 0, Flag<false>{});
+        p_chunk(rb, 1, Flag<false>{});
+      }
       tmem_st16(tSh, *reinterpret_cast<const uint32_t(*)[16]>(pk));
       tmem_st16(tSh + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
       tmem_wait_st();

@@ -305,6 +305,13 @@ __device__ __forceinline__ void ex2_fma2(float x0, float x1, float& y0, float& y
   y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+// A compile-time flag for a code path chosen once per tile (say, a tile that needs the causal
+// mask), so that the common path carries no per-element tests.
+template <bool B>
+struct Flag {
+  static constexpr bool value = B;
+};
+
 // Pack two floats into bf16x2 (round to nearest even); `lo` lands in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
