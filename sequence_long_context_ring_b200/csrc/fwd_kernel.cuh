@@ -507,86 +507,97 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int lim = kvi.kv_end(p) - kv0;
       if (p.causal) lim = min(lim, q_row - kv0 + 1);
       const bool masked = __any_sync(0xffffffffu, lim < kBN);
-      const bool emu = !masked;
+      // The rest of the tile, instantiated with and without the mask code: only tiles at the
+      // diagonal or at a ragged chunk end take the masked instance, the others carry no
+      // per-element tests.
+      auto tile = [&](auto with_mask) {
+        constexpr bool kMasked = decltype(with_mask)::value;
+        const bool emu = !kMasked;
 
-      // The whole S row stays in registers until the tile is settled (a rare recompute needs
-      // it; P overwrites the first 64 columns of S in TMEM).  Chunks 2 and 3 load while the
-      // exponentials of chunks 0 and 1 run.
-      uint32_t ra[32], rb[32], rc[32], rd[32];
-      tmem_ld32(tS + 0, ra);
-      tmem_ld32(tS + 32, rb);
-      tmem_wait_ld();
-      tmem_ld32(tS + 64, rc);
-      tmem_ld32(tS + 96, rd);
-      if (masked) {
-        mask_chunk(ra, 0, lim);
-        mask_chunk(rb, 32, lim);
-      }
-      if (i == 0) {
-        // first tile: the exact row max before any exponential
+        // The whole S row stays in registers until the tile is settled (a rare recompute needs
+        // it; P overwrites the first 64 columns of S in TMEM).  Chunks 2 and 3 load while the
+        // exponentials of chunks 0 and 1 run.
+        uint32_t ra[32], rb[32], rc[32], rd[32];
+        tmem_ld32(tS + 0, ra);
+        tmem_ld32(tS + 32, rb);
         tmem_wait_ld();
-        if (masked) {
-          mask_chunk(rc, 64, lim);
-          mask_chunk(rd, 96, lim);
+        tmem_ld32(tS + 64, rc);
+        tmem_ld32(tS + 96, rd);
+        if constexpr (kMasked) {
+          mask_chunk(ra, 0, lim);
+          mask_chunk(rb, 32, lim);
         }
-        m_run = fmaxf(fmaxf(max_chunk(ra), max_chunk(rb)), fmaxf(max_chunk(rc), max_chunk(rd))) * sl2;
-      }
-      uint64_t negm2;
-      {
-        const float m_off = (m_run == -INFINITY) ? 0.f : m_run;
-        negm2 = f2_pack(-m_off, -m_off);
-      }
-      float l_tile = exp_chunk(ra, 0, negm2, emu);
-      l_tile += exp_chunk(rb, 1, negm2, emu);
-      if (i > 0) {
-        tmem_wait_ld();
-        if (masked) {
-          mask_chunk(rc, 64, lim);
-          mask_chunk(rd, 96, lim);
+        if (i == 0) {
+          // first tile: the exact row max before any exponential
+          tmem_wait_ld();
+          if constexpr (kMasked) {
+            mask_chunk(rc, 64, lim);
+            mask_chunk(rd, 96, lim);
+          }
+          m_run = fmaxf(fmaxf(max_chunk(ra), max_chunk(rb)), fmaxf(max_chunk(rc), max_chunk(rd))) * sl2;
         }
-      }
-      // Before the first half of P is released: the offset must keep every exponential of the
-      // tile below 2^kStaleLimit (keys [0,64) by their sum, [64,128) by their max).
-      const float m23 = fmaxf(max_chunk(rc), max_chunk(rd)) * sl2;
-      const bool over = !(l_tile <= kStaleLimitPow) || m23 > m_run + kStaleLimit;
-      if (__any_sync(0xffffffffu, over)) {
-        // rare: move the offset of the rows that need it to their tile max, rescale O and l
-        // (O holds the previous tiles' sum: PV of the previous tile has completed because S of
-        // this tile was issued after it), and recompute the whole tile's P; rows whose offset
-        // did not move recompute the same values
-        float alpha = 1.f;
-        if (over) {
-          const float m_new = fmaxf(fmaxf(max_chunk(ra), max_chunk(rb)) * sl2, m23);
-          if (m_new > m_run) {
-            alpha = ex2_approx(m_run - m_new);  // 0 when m_run = -inf
-            m_run = m_new;
+        uint64_t negm2;
+        {
+          const float m_off = (m_run == -INFINITY) ? 0.f : m_run;
+          negm2 = f2_pack(-m_off, -m_off);
+        }
+        float l_tile = exp_chunk(ra, 0, negm2, emu);
+        l_tile += exp_chunk(rb, 1, negm2, emu);
+        if (i > 0) {
+          tmem_wait_ld();
+          if constexpr (kMasked) {
+            mask_chunk(rc, 64, lim);
+            mask_chunk(rd, 96, lim);
           }
         }
-        const float m_off = (m_run == -INFINITY) ? 0.f : m_run;
-        negm2 = f2_pack(-m_off, -m_off);
-        tmem_wait_st();
-        l_tile = exp_chunk(ra, 0, negm2, false);
-        l_tile += exp_chunk(rb, 1, negm2, false);
-        l_tile += exp_chunk(rc, 2, negm2, false);
-        l_tile += exp_chunk(rd, 3, negm2, false);
-        l_run = l_run * alpha + l_tile;
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t r[32];
-          tmem_ld32(tO + cc * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(tO + cc * 32, r);
+        // Before the first half of P is released: the offset must keep every exponential of the
+        // tile below 2^kStaleLimit (keys [0,64) by their sum, [64,128) by their max).
+        const float m23 = fmaxf(max_chunk(rc), max_chunk(rd)) * sl2;
+        const bool over = !(l_tile <= kStaleLimitPow) || m23 > m_run + kStaleLimit;
+        if (__any_sync(0xffffffffu, over)) {
+          // rare: move the offset of the rows that need it to their tile max, rescale O and l
+          // (O holds the previous tiles' sum: PV of the previous tile has completed because S of
+          // this tile was issued after it), and recompute the whole tile's P; rows whose offset
+          // did not move recompute the same values
+          float alpha = 1.f;
+          if (over) {
+            const float m_new = fmaxf(fmaxf(max_chunk(ra), max_chunk(rb)) * sl2, m23);
+            if (m_new > m_run) {
+              alpha = ex2_approx(m_run - m_new);  // 0 when m_run = -inf
+              m_run = m_new;
+            }
+          }
+          const float m_off = (m_run == -INFINITY) ? 0.f : m_run;
+          negm2 = f2_pack(-m_off, -m_off);
+          tmem_wait_st();
+          l_tile = exp_chunk(ra, 0, negm2, false);
+          l_tile += exp_chunk(rb, 1, negm2, false);
+          l_tile += exp_chunk(rc, 2, negm2, false);
+          l_tile += exp_chunk(rd, 3, negm2, false);
+          l_run = l_run * alpha + l_tile;
+  #pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld32(tO + cc * 32, r);
+            tmem_wait_ld();
+  #pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(tO + cc * 32, r);
+          }
+          publish(&p_half[ab]);
+          publish(&p_full[ab]);
+        } else {
+          publish(&p_half[ab]);
+          l_tile += exp_chunk(rc, 2, negm2, emu);
+          l_tile += exp_chunk(rd, 3, negm2, emu);
+          l_run += l_tile;
+          publish(&p_full[ab]);
         }
-        publish(&p_half[ab]);
-        publish(&p_full[ab]);
+      };
+      if (masked) {
+        tile(Flag<true>{});
       } else {
-        publish(&p_half[ab]);
-        l_tile += exp_chunk(rc, 2, negm2, emu);
-        l_tile += exp_chunk(rd, 3, negm2, emu);
-        l_run += l_tile;
-        publish(&p_full[ab]);
+        tile(Flag<false>{});
       }
     }
 
