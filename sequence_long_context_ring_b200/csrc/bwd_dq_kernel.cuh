@@ -19,7 +19,9 @@
 // S(i) goes to buffer i&1; dS(i) of keys [64h, 64h+64) (bf16, two per column) overwrites
 // columns [64h, 64h+32) of it, which warpgroup h has already read.
 // Per iteration the MMA issues S(i+1) and dP(i+1) before dQ += dS(i) K(i), so the tensor pipe
-// computes the next tile's products while the elementwise warps work on this one.
+// computes the next tile's products while the elementwise warps work on this one.  The warps
+// turn S(i) into P(i) as soon as S(i) lands, before dP(i) (issued only once they have read
+// dP(i-1)) arrives.
 #pragma once
 #include "sm100.cuh"
 
@@ -346,6 +348,31 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       uint32_t sa[32], sb[32];
       tmem_ld32(tS + 0, sa);
       tmem_ld32(tS + 32, sb);
+      tmem_wait_ld();
+      // P = 2^(S * scale * log2(e) - LSE * log2(e)) of one 32-key chunk, in place (fp32 bits),
+      // computed while dP(i) is still on its way; the mask code exists only in the masked
+      // instance
+      auto p_chunk = [&](uint32_t (&r)[32], int cc, auto with_mask) {
+        if constexpr (decltype(with_mask)::value) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (cc * 32 + e >= lim) r[e] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * e2]), __uint_as_float(r[2 * e2 + 1])), sl2x2, nl2), x0, x1);
+          r[2 * e2] = __float_as_uint(ex2_approx(x0));
+          r[2 * e2 + 1] = __float_as_uint(ex2_approx(x1));
+        }
+      };
+      if (masked) {
+        p_chunk(sa, 0, Flag<true>{});
+        p_chunk(sb, 1, Flag<true>{});
+      } else {
+        p_chunk(sa, 0, Flag<false>{});
+        p_chunk(sb, 1, Flag<false>{});
+      }
       if (!__all_sync(0xffffffffu, wait_bounded(&dp_full[i & 1], (i >> 1) & 1, ctl, kQSiteDp))) { ok = false; break; }
       tc_fence_after();
       uint32_t dpa[32], dpb[32];
@@ -356,40 +383,20 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dp_free);
-      // dS of one 32-key chunk -> 16 packed bf16 columns; the mask code exists only in the
-      // masked instance
-      auto ds_chunk = [&](uint32_t (&r)[32], const uint32_t (&g)[32], int cc, auto with_mask) {
-        if constexpr (decltype(with_mask)::value) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (cc * 32 + e >= lim) r[e] = __float_as_uint(-INFINITY);
-        }
+      // dS = P (dP - D) of one 32-key chunk -> 16 packed bf16 columns over S
+      auto ds_chunk = [&](const uint32_t (&pr)[32], const uint32_t (&g)[32], int cc) {
         uint32_t pk[16];
-        // every exponential of the chunk first, then dS = P (dP - D) and the bf16 packs
-        float pv[32];
-#pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * e2]), __uint_as_float(r[2 * e2 + 1])), sl2x2, nl2), x0, x1);
-          pv[2 * e2] = ex2_approx(x0);
-          pv[2 * e2 + 1] = ex2_approx(x1);
-        }
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
           const uint64_t dd = f2_add(f2_pack(__uint_as_float(g[2 * e2]), __uint_as_float(g[2 * e2 + 1])), nD2);
           float d0, d1;
-          f2_unpack(f2_mul(f2_pack(pv[2 * e2], pv[2 * e2 + 1]), dd), d0, d1);
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(pr[2 * e2]), __uint_as_float(pr[2 * e2 + 1])), dd), d0, d1);
           pk[e2] = pack_bf16x2(d0, d1);
         }
         tmem_st16(tS + cc * 16, pk);
       };
-      if (masked) {
-        ds_chunk(sa, dpa, 0, Flag<true>{});
-        ds_chunk(sb, dpb, 1, Flag<true>{});
-      } else {
-        ds_chunk(sa, dpa, 0, Flag<false>{});
-        ds_chunk(sb, dpb, 1, Flag<false>{});
-      }
+      ds_chunk(sa, dpa, 0);
+      ds_chunk(sb, dpb, 1);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

@@ -26,7 +26,9 @@
 // that warpgroup has already read; dS^T likewise over dP^T.
 // MMA order per query tile i: dV(i), S^T(i+1), dK(i), dP^T(i+1).  S^T(i+1) may overwrite the
 // S^T columns as soon as dV(i) has been issued (the tensor pipe runs one thread's MMAs in
-// order), so the warps compute P(i+1) while the tensor cores run dK(i) and dP^T(i+1).
+// order), so the warps compute P(i+1) while the tensor cores run dK(i) and dP^T(i+1).  Each
+// warp releases its P^T in two 32-column halves, and dV(i) runs on the first halves (queries
+// [0,32) and [64,96)) while the second halves are being computed.
 // Shared memory holds, per Q/dO stage, -LSE * log2(e) and D of the tile's 128 queries: the
 // warps read them as broadcast 16-byte vectors.
 #pragma once
@@ -165,6 +167,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* dp_full = bars + 6;
   uint64_t* p_full = bars + 7;
   uint64_t* ds_full = bars + 8;
+  uint64_t* p_half = bars + 9;     // the first 32 columns of each warpgroup's P^T are in TMEM
   uint64_t* done_bar = bars + 11;
   uint64_t* drain_bar = bars + 12;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
@@ -184,6 +187,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, 8);
+    mbar_init(p_half, 8);
     mbar_init(ds_full, 8);
     mbar_init(done_bar, 1);
     mbar_init(drain_bar, 1);
@@ -305,14 +309,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       for (int i = 0; i < it.n_iter && ok; ++i) {
         const int st = i & 1;
-        // (1) dV += P^T dO  [A = P^T in TMEM (keys x queries), B = dO N-major]
-        if (!wait_bounded(p_full, i & 1, ctl, kBSiteMmaP)) { ok = false; break; }
-        tc_fence_after();
+        // (1) dV += P^T dO  [A = P^T in TMEM (keys x queries), B = dO N-major], in two halves:
+        // queries [0,32) and [64,96) once each warpgroup has stored its first chunk, then the rest
         {
           const uint32_t b = stage(do_n0, i);
+          if (!wait_bounded(p_half, i & 1, ctl, kBSiteMmaP)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk)
-            umma_ts(tDV, tS + bwd_a_col(kk), sdesc_lo_at(b, kk * 2048), idesc_tn, (i > 0 || kk > 0));
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int kk = (q4 >> 1) * 4 + (q4 & 1);   // 0, 1, 4, 5
+            umma_ts(tDV, tS + bwd_a_col(kk), sdesc_lo_at(b, kk * 2048), idesc_tn, (i > 0 || q4 > 0));
+          }
+          if (!wait_bounded(p_full, i & 1, ctl, kBSiteMmaP)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int kk = (q4 >> 1) * 4 + (q4 & 1) + 2;   // 2, 3, 6, 7
+            umma_ts(tDV, tS + bwd_a_col(kk), sdesc_lo_at(b, kk * 2048), idesc_tn, 1u);
+          }
         }
         // (2) S^T(i+1) over P^T(i) (read by dV(i), issued before)
         const bool more = i + 1 < it.n_iter;
@@ -402,19 +416,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pk[c >> 1] = pack_bf16x2(p0, p1);
         }
       };
+      // each chunk is released as soon as it is stored, so dV(i) starts on the first half
+      auto release = [&](int cc, uint64_t* bar) {
+        tmem_st16(tSh + 16 * cc, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16 * cc));
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar);
+      };
       if (masked) {
         p_chunk(ra, 0, Flag<true>{});
+        release(0, p_half);
         p_chunk(rb, 1, Flag<true>{});
       } else {
         p_chunk(ra, 0, Flag<false>{});
+        release(0, p_half);
         p_chunk(rb, 1, Flag<false>{});
       }
-      tmem_st16(tSh, *reinterpret_cast<const uint32_t(*)[16]>(pk));
-      tmem_st16(tSh + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      release(1, p_full);
 
       if (!__all_sync(0xffffffffu, wait_bounded(dp_full, i & 1, ctl, kBSiteSoftDp))) { ok = false; break; }
       tc_fence_after();
