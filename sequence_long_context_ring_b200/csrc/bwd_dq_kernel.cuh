@@ -11,17 +11,20 @@
 // Warp roles (320 threads):
 //   warps 0-7  elementwise: warp w handles query rows 32(w%4) .. +31 (thread <-> TMEM lane)
 //              and keys [64(w/4), 64(w/4) + 64) -- no row reduction is needed (LSE and D are
-//              known), so the two warpgroups split the columns; epilogue writes dQ (each
-//              warpgroup half of the d columns)
-//   warp  8    loads: Q and dO once; K_i into a 3-slot ring, V_i into a 2-slot ring (TMA)
+//              known), so the two warpgroups split the columns.  Before the loop they copy the
+//              tile's Q (warpgroup 0) and dO (warpgroup 1) rows into TMEM, where they serve as
+//              the A operand of every S and dP MMA; the epilogue writes dQ (each warpgroup half
+//              of the d columns)
+//   warp  8    loads: K_i into a 4-slot ring, V_i into a 3-slot ring (TMA)
 //   warp  9    MMA issuer (one thread)
-// TMEM columns: dQ [0,128)  S buffer 0 [128,256)  S buffer 1 [256,384)  dP [384,512).
-// S(i) goes to buffer i&1; dS(i) of keys [64h, 64h+64) (bf16, two per column) overwrites
-// columns [64h, 64h+32) of it, which warpgroup h has already read.
-// Per iteration the MMA issues S(i+1) and dP(i+1) before dQ += dS(i) K(i), so the tensor pipe
-// computes the next tile's products while the elementwise warps work on this one.  The warps
-// turn S(i) into P(i) as soon as S(i) lands, before dP(i) (issued only once they have read
-// dP(i-1)) arrives.
+// TMEM columns: dQ [0,128)  S [128,256)  dP [256,384)  Q [384, 384+d/2)  dO [384+d/2, 384+d)
+// (Q and dO as bf16 pairs, one row per lane).  S and dP take their A operand from TMEM, so each
+// of their MMAs reads only the K or V tile from shared memory.  dS of keys [64h, 64h+64)
+// (bf16, two per column) overwrites dP columns [64h, 64h+32), which warpgroup h has already
+// read.
+// Per iteration i: S(i+1) is issued as soon as the warps hold S(i) in registers; dQ(i) once
+// dS(i) is in TMEM; then dP(i+1) over dS(i) (the pipe runs one thread's MMAs in order).  The
+// warps turn S(i) into P(i) while dQ(i-1) and dP(i) run on the tensor cores.
 #pragma once
 #include "sm100.cuh"
 
@@ -30,16 +33,13 @@ namespace cpattn {
 constexpr int kDqThreads = 320;
 constexpr int kDqLoadWarp = 8;
 constexpr int kDqMmaWarp = 9;
-#ifndef CPATTN_DQ_KSLOTS
-#define CPATTN_DQ_KSLOTS 3
-#endif
-// K_i is read by S(i) (issued one iteration early) and by dQ(i): it holds its slot about two
-// iterations, V_i (read by dP(i) only) about one, so K gets more of the five slots.
-constexpr int kDqKSlots = CPATTN_DQ_KSLOTS;
-constexpr int kDqVSlots = 5 - kDqKSlots;
+// K_i is read by S(i) (issued most of an iteration early) and by dQ(i), V_i by dP(i) only, so
+// K gets more of the seven slots.
+constexpr int kDqKSlots = 4;
+constexpr int kDqVSlots = 3;
 
 enum DqSite : int {
-  kQSiteLoadK = 33, kQSiteLoadV = 34, kQSiteMmaQ = 35, kQSiteMmaK = 36, kQSiteMmaV = 37, kQSiteMmaDpFree = 38,
+  kQSiteLoadK = 33, kQSiteLoadV = 34, kQSiteMmaQ = 35, kQSiteMmaK = 36, kQSiteMmaV = 37, kQSiteMmaSFree = 38,
   kQSiteMmaDs = 39, kQSiteS = 40, kQSiteDp = 41, kQSiteDone = 42, kQSiteDrain = 43,
 };
 
@@ -52,11 +52,15 @@ struct DqParams {
   const float* lse;   // [B, Hq, L] natural-log LSE of the forward
   long long lse_sb, lse_sh, lse_sl;
   const float* Dvec;  // [B, Hq, L] rowsum(dO * O), contiguous
+  const __nv_bfloat16* q;    // [B, Hq, L, d] by the strides below (rows d-contiguous)
+  long long q_sb, q_sh, q_sl;
+  const __nv_bfloat16* dout;
+  long long do_sb, do_sh, do_sl;
   __nv_bfloat16* dq;  // [B, Hq, L, d] by the strides below
   long long dq_sb, dq_sh, dq_sl;
   int* status;
   unsigned long long wait_limit_ns;
-  int debug_fault;    // 3: the load warp skips the Q/dO tile load (a test of the timeout path)
+  int debug_fault;    // 3: the warps never report Q/dO in TMEM (a test of the timeout path)
 };
 
 struct DqItem {
@@ -114,16 +118,15 @@ __device__ __forceinline__ void dq_wait_drain(uint64_t* bar, uint32_t parity, co
   }
 }
 
-// Dynamic shared memory: 1 KB alignment slack + Q + dO + 3 K slots + 2 V slots + barriers
+// Dynamic shared memory: 1 KB alignment slack + 4 K slots + 3 V slots + barriers
 // (d = 128: 230,656 bytes).
 __host__ __device__ constexpr size_t bwd_dq_smem_bytes(int d) {
-  return 1024 + static_cast<size_t>(2 + kDqKSlots + kDqVSlots) * 128 * d * 2 + 256;
+  return 1024 + static_cast<size_t>(kDqKSlots + kDqVSlots) * 128 * d * 2 + 256;
 }
 
 template <int D>
 __global__ void __launch_bounds__(kDqThreads, 1)
-    ring_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+    ring_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const DqParams p) {
   static_assert(D == 64 || D == 128, "head dim");
   constexpr int kBoxes = D / 64;
@@ -132,29 +135,29 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_s = smem;
-  uint8_t* do_s = smem + kTile;
-  uint8_t* k_s = smem + 2 * kTile;                  // [kDqKSlots]
+  uint8_t* k_s = smem;                              // [kDqKSlots]
   uint8_t* v_s = k_s + kDqKSlots * kTile;           // [kDqVSlots]
   uint64_t* bars = reinterpret_cast<uint64_t*>(v_s + kDqVSlots * kTile);
   // Barriers (a waiter on a two-barrier pair [t & 1] uses parity (t >> 1) & 1; none can run two
   // phases ahead of its waiter, because each next phase needs that waiter's own progress):
-  //  q_full          Q and dO landed
+  //  qa_full         elementwise -> MMA: Q and dO rows in TMEM (8 warp arrivals)
   //  k_full[kK]      K_i landed in slot i % kK (parity (i / kK) & 1)
   //  v_full[kV]      V_i landed in slot i % kV (parity (i / kV) & 1)
   //  k_free[kK]      MMA commit after dQ(i): slot i % kK (K_i) no longer read
-  //  s_full[2]       MMA commit after S(i) (buffer i & 1)
-  //  dp_full[2]      MMA commit after dP(i): dP(i) in TMEM, and V_i no longer read
-  //  dp_free         elementwise -> MMA: dP(i) loaded into registers (8 warp arrivals)
+  //  v_free[kV]      MMA commit after dP(i): slot i % kV (V_i) no longer read
+  //  s_full          MMA commit after S(i) (parity i & 1)
+  //  s_free          elementwise -> MMA: S(i) loaded into registers (8 warp arrivals)
+  //  dp_full[2]      MMA commit after dP(i)
   //  ds_full[2]      elementwise -> MMA: dS(i) written to TMEM (8 warp arrivals)
-  uint64_t* q_full = bars + 0;
+  uint64_t* qa_full = bars + 0;
   uint64_t* k_full = bars + 1;                      // [kK]
   uint64_t* v_full = k_full + kDqKSlots;            // [kV]
   uint64_t* k_free = v_full + kDqVSlots;            // [kK]
-  uint64_t* s_full = k_free + kDqKSlots;            // [2]
-  uint64_t* dp_full = s_full + 2;                   // [2]
-  uint64_t* dp_free = dp_full + 2;
-  uint64_t* ds_full = dp_free + 1;                  // [2]
+  uint64_t* v_free = k_free + kDqKSlots;            // [kV]
+  uint64_t* s_full = v_free + kDqVSlots;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* dp_full = s_free + 1;                   // [2]
+  uint64_t* ds_full = dp_full + 2;                  // [2]
   uint64_t* drain_bar = ds_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -165,18 +168,21 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(qa_full, 8);
     for (int s = 0; s < kDqKSlots; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_free[s], 1);
     }
-    for (int s = 0; s < kDqVSlots; ++s) mbar_init(&v_full[s], 1);
+    for (int s = 0; s < kDqVSlots; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_free[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 8);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
       mbar_init(&dp_full[s], 1);
       mbar_init(&ds_full[s], 8);
     }
-    mbar_init(dp_free, 8);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     *skip_flag = (p.status != nullptr && *reinterpret_cast<volatile int*>(p.status) != 0) ? 1 : 0;
@@ -194,26 +200,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const DqItem it = decode_dq_item(p);
   const int T = it.n_tiles;
-  const uint32_t tDQ = tmem_base, tS0 = tmem_base + 128, tDP = tmem_base + 384;
+  const uint32_t tDQ = tmem_base, tS = tmem_base + 128, tDP = tmem_base + 256;
+  const uint32_t tQa = tmem_base + 384, tDOa = tmem_base + 384 + D / 2;
 
   if (warp == kDqLoadWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_do);
       const uint64_t pol_kv = policy_evict_last();
-      const uint64_t pol_q = policy_evict_first();
-      const bool load_q = (p.debug_fault != 3);
-      if (load_q) {
-        mbar_arrive_expect_tx(q_full, 2 * kTile);
-#pragma unroll
-        for (int x = 0; x < kBoxes; ++x) {
-          tma_load_4d(q_s + x * kBoxBytes, &tm_q, q_full, x * 64, it.row0, it.h, it.b, pol_q);
-          tma_load_4d(do_s + x * kBoxBytes, &tm_do, q_full, x * 64, it.row0, it.h, it.b, pol_q);
-        }
-      }
       int nk = 0, nv = 0;  // loads issued
       DqKvIter kvi(p, it);
       for (int i = 0; i < T; ++i, kvi.next(p)) {
@@ -229,10 +224,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           for (int x = 0; x < kBoxes; ++x) tma_load_4d(dst + x * kBoxBytes, &tm_k, full, x * 64, kv0, it.g, it.b, pol_kv);
           ++nk;
         }
-        // V_i takes the slot of V_{i-kV}: free once dP(i-kV) completed (dp_full of that tile;
-        // it cannot run two phases ahead: dP(i) needs V_i)
-        if (i >= kDqVSlots && !wait_bounded(&dp_full[(i - kDqVSlots) & 1], ((i - kDqVSlots) >> 1) & 1, ctl,
-                                            kQSiteLoadV)) break;
+        // V_i takes the slot of V_{i-kV}: free once dP(i-kV) completed
+        if (i >= kDqVSlots &&
+            !wait_bounded(&v_free[i % kDqVSlots], ((i / kDqVSlots) - 1) & 1, ctl, kQSiteLoadV)) break;
         {
           uint64_t* full = &v_full[i % kDqVSlots];
           uint8_t* dst = v_s + (i % kDqVSlots) * kTile;
@@ -243,7 +237,6 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
       }
       // drain: every load this thread issued has landed before the CTA can exit
-      if (load_q) dq_wait_drain(q_full, 0, ctl);
       for (int n = (nk > kDqKSlots ? nk - kDqKSlots : 0); n < nk; ++n)
         dq_wait_drain(&k_full[n % kDqKSlots], (n / kDqKSlots) & 1, ctl);
       for (int n = (nv > kDqVSlots ? nv - kDqVSlots : 0); n < nv; ++n)
@@ -253,19 +246,19 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   } else if (warp == kDqMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc_kk = make_idesc_bf16(128, 128, false);  // S, dP: A and B K-major
+      constexpr uint32_t idesc_kk = make_idesc_bf16(128, 128, false);  // S, dP: A TMEM, B K-major
       constexpr uint32_t idesc_o = make_idesc_bf16(128, D, true);      // dQ: A TMEM, B (K) N-major
-      // Operand descriptors, built once: Q, dO, and slot 0 of K and V as K-major tiles, slot 0 of K
-      // as the N-major B of dQ; a slot's descriptor is slot 0's plus the slot offset.
-      const uint32_t q_d = sdesc_lo(smem_u32(q_s), 16), do_d = sdesc_lo(smem_u32(do_s), 16);
+      // Operand descriptors, built once: slot 0 of K and V as K-major tiles, slot 0 of K as the
+      // N-major B of dQ; a slot's descriptor is slot 0's plus the slot offset.
       const uint32_t k_d0 = sdesc_lo(smem_u32(k_s), 16), v_d0 = sdesc_lo(smem_u32(v_s), 16);
       const uint32_t kn_d0 = sdesc_lo(smem_u32(k_s), kBoxBytes);
-      // X = A B^T over d (both tiles d-contiguous), 128 x 128 into TMEM column d_tmem
-      auto issue_kk = [=](uint32_t d_tmem, uint32_t a, uint32_t b) {
+      // X = A B^T over d: A (Q or dO rows) from TMEM, 8 columns per 16 d; B d-contiguous in
+      // shared memory; 128 x 128 into TMEM column d_tmem
+      auto issue_kk = [=](uint32_t d_tmem, uint32_t a_tmem, uint32_t b) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          umma_ss(d_tmem, sdesc_lo_at(a, off), sdesc_lo_at(b, off), idesc_kk, kk > 0 ? 1u : 0u);
+          umma_ts(d_tmem, a_tmem + 8u * kk, sdesc_lo_at(b, off), idesc_kk, kk > 0 ? 1u : 0u);
         }
       };
       auto wait_k = [&](int i) { return wait_bounded(&k_full[i % kDqKSlots], (i / kDqKSlots) & 1, ctl, kQSiteMmaK); };
@@ -274,43 +267,45 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       };
       auto kdesc = [&](int i) { return sdesc_lo_at(k_d0, (i % kDqKSlots) * kTile); };
       auto vdesc = [&](int i) { return sdesc_lo_at(v_d0, (i % kDqVSlots) * kTile); };
+      // dP(i) into the dP columns; V_i's slot is free once it completes
+      auto issue_dp = [&](int i) -> bool {
+        if (!wait_v(i)) return false;
+        issue_kk(tDP, tDOa, vdesc(i));
+        umma_commit(&dp_full[i & 1]);
+        umma_commit(&v_free[i % kDqVSlots]);
+        return true;
+      };
 
-      bool ok = wait_bounded(q_full, 0, ctl, kQSiteMmaQ);
+      bool ok = wait_bounded(qa_full, 0, ctl, kQSiteMmaQ);
       if (ok && T > 0) {
+        tc_fence_after();
         ok = wait_k(0);
         if (ok) {
-          issue_kk(tS0, q_d, kdesc(0));
-          umma_commit(&s_full[0]);
-          ok = wait_v(0);
-        }
-        if (ok) {
-          issue_kk(tDP, do_d, vdesc(0));
-          umma_commit(&dp_full[0]);
+          issue_kk(tS, tQa, kdesc(0));
+          umma_commit(s_full);
+          ok = issue_dp(0);
         }
       }
       for (int i = 0; i < T && ok; ++i) {
+        // S(i+1) over S(i), once the elementwise warps hold S(i) in registers
         if (i + 1 < T) {
-          // S(i+1) into buffer (i+1)&1, which held dS(i-1): dQ(i-1) was issued before
+          if (!wait_bounded(s_free, i & 1, ctl, kQSiteMmaSFree)) { ok = false; break; }
           if (!wait_k(i + 1)) { ok = false; break; }
-          issue_kk(tS0 + ((i + 1) & 1) * 128, q_d, kdesc(i + 1));
-          umma_commit(&s_full[(i + 1) & 1]);
-          // dP(i+1) over dP(i), once the elementwise warps hold dP(i) in registers
-          if (!wait_v(i + 1)) { ok = false; break; }
-          if (!wait_bounded(dp_free, i & 1, ctl, kQSiteMmaDpFree)) { ok = false; break; }
           tc_fence_after();
-          issue_kk(tDP, do_d, vdesc(i + 1));
-          umma_commit(&dp_full[(i + 1) & 1]);
+          issue_kk(tS, tQa, kdesc(i + 1));
+          umma_commit(s_full);
         }
         // dQ += dS(i) K(i): A = dS from TMEM (8 columns per 16 keys), B = K N-major
         if (!wait_bounded(&ds_full[i & 1], (i >> 1) & 1, ctl, kQSiteMmaDs)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t ds_t = tS0 + (i & 1) * 128;
         const uint32_t kn = sdesc_lo_at(kn_d0, (i % kDqKSlots) * kTile);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // keys [16 kk, 16 kk + 16): written by warpgroup kk / 4
-          umma_ts(tDQ, ds_t + 64u * (kk >> 2) + 8u * (kk & 3), sdesc_lo_at(kn, kk * 2048), idesc_o,
+          umma_ts(tDQ, tDP + 64u * (kk >> 2) + 8u * (kk & 3), sdesc_lo_at(kn, kk * 2048), idesc_o,
                   (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&k_free[i % kDqKSlots]);
+        // dP(i+1) over dS(i), which dQ(i) (issued before it) reads
+        if (i + 1 < T && !issue_dp(i + 1)) { ok = false; break; }
       }
       // drain: all MMAs issued by this thread are complete before TMEM is freed
       umma_commit(drain_bar);
@@ -324,6 +319,32 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const uint32_t lofs = (quarter * 32u) << 16;
     const int q_row = it.row0 + static_cast<int>(quarter * 32 + lane);
     const bool q_live = q_row < it.q_end;
+    // This row of Q (warpgroup 0) or dO (warpgroup 1) into TMEM as bf16 pairs: the A operand of
+    // S = Q K^T and dP = dO V^T.  Rows past the sequence are zeros; rows past the chunk are
+    // read but get probability 0 below.
+    {
+      const __nv_bfloat16* src = hh == 0 ? p.q + it.b * p.q_sb + it.h * p.q_sh + static_cast<long long>(q_row) * p.q_sl
+                                         : p.dout + it.b * p.do_sb + it.h * p.do_sh + static_cast<long long>(q_row) * p.do_sl;
+      const bool in_seq = q_row < p.L;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint4 x = make_uint4(0u, 0u, 0u, 0u);
+          if (in_seq) x = *reinterpret_cast<const uint4*>(src + c * 64 + v * 8);
+          r[4 * v] = x.x;
+          r[4 * v + 1] = x.y;
+          r[4 * v + 2] = x.z;
+          r[4 * v + 3] = x.w;
+        }
+        tmem_st32((hh == 0 ? tQa : tDOa) + lofs + c * 32, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0 && p.debug_fault != 3) mbar_arrive(qa_full);
+    }
     // rows past the chunk (ragged tail) get LSE = +inf: probability 0, no contribution
     float lse2 = INFINITY, Dr = 0.f;
     if (q_live) {
@@ -338,17 +359,21 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     bool ok = true;
     DqKvIter kvi(p, it);
     for (int i = 0; i < T; ++i, kvi.next(p)) {
-      const uint32_t tS = tS0 + (i & 1) * 128 + lofs + hh * 64;
+      const uint32_t tSh = tS + lofs + hh * 64, tDPh = tDP + lofs + hh * 64;
       const int kv0 = kvi.kv0(p) + hh * 64;  // first key of this warp's half
       int lim = kvi.kv_end(p) - kv0;
       if (p.causal) lim = min(lim, q_row - kv0 + 1);
       const bool masked = __any_sync(0xffffffffu, lim < 64);
-      if (!__all_sync(0xffffffffu, wait_bounded(&s_full[i & 1], (i >> 1) & 1, ctl, kQSiteS))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, wait_bounded(s_full, i & 1, ctl, kQSiteS))) { ok = false; break; }
       tc_fence_after();
       uint32_t sa[32], sb[32];
-      tmem_ld32(tS + 0, sa);
-      tmem_ld32(tS + 32, sb);
+      tmem_ld32(tSh + 0, sa);
+      tmem_ld32(tSh + 32, sb);
       tmem_wait_ld();
+      // S(i) is in registers: the MMA may write S(i+1)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
       // P = 2^(S * scale * log2(e) - LSE * log2(e)) of one 32-key chunk, in place (fp32 bits),
       // computed while dP(i) is still on its way; the mask code exists only in the masked
       // instance
@@ -376,14 +401,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       if (!__all_sync(0xffffffffu, wait_bounded(&dp_full[i & 1], (i >> 1) & 1, ctl, kQSiteDp))) { ok = false; break; }
       tc_fence_after();
       uint32_t dpa[32], dpb[32];
-      tmem_ld32(tDP + lofs + hh * 64, dpa);
-      tmem_ld32(tDP + lofs + hh * 64 + 32, dpb);
+      tmem_ld32(tDPh, dpa);
+      tmem_ld32(tDPh + 32, dpb);
       tmem_wait_ld();
-      // dP(i) is in registers: the MMA may write dP(i+1)
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dp_free);
-      // dS = P (dP - D) of one 32-key chunk -> 16 packed bf16 columns over S
+      // dS = P (dP - D) of one 32-key chunk -> 16 packed bf16 columns over dP (already read)
       auto ds_chunk = [&](const uint32_t (&pr)[32], const uint32_t (&g)[32], int cc) {
         uint32_t pk[16];
 #pragma unroll
@@ -393,7 +414,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           f2_unpack(f2_mul(f2_pack(__uint_as_float(pr[2 * e2]), __uint_as_float(pr[2 * e2 + 1])), dd), d0, d1);
           pk[e2] = pack_bf16x2(d0, d1);
         }
-        tmem_st16(tS + cc * 16, pk);
+        tmem_st16(tDPh + cc * 16, pk);
       };
       ds_chunk(sa, dpa, 0);
       ds_chunk(sb, dpb, 1);

@@ -251,13 +251,13 @@ cp_status_t launch_bwd_d(const BwdParams& p, const CUtensorMap& mq, const CUtens
 }
 
 template <int D>
-cp_status_t launch_bwd_dq_d(const DqParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                            const CUtensorMap& mdo, int64_t grid, cudaStream_t s) {
+cp_status_t launch_bwd_dq_d(const DqParams& p, const CUtensorMap& mk, const CUtensorMap& mv, int64_t grid,
+                            cudaStream_t s) {
   const size_t smem = bwd_dq_smem_bytes(D);
   if (cudaFuncSetAttribute(ring_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return CP_ERR_CUDA;
-  ring_bwd_dq_kernel<D><<<(unsigned)grid, kDqThreads, smem, s>>>(mq, mk, mv, mdo, p);
+  ring_bwd_dq_kernel<D><<<(unsigned)grid, kDqThreads, smem, s>>>(mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
@@ -425,6 +425,15 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
   qp.lse_sh = p.lse_sh;
   qp.lse_sl = p.lse_sl;
   qp.Dvec = Dvec;
+  // Q and dO rows, read by the kernel's elementwise warps into TMEM (the same views as the maps)
+  qp.q = static_cast<const __nv_bfloat16*>(vq.data);
+  qp.q_sb = vq.sB;
+  qp.q_sh = vq.sH;
+  qp.q_sl = vq.sL;
+  qp.dout = static_cast<const __nv_bfloat16*>(vdo.data);
+  qp.do_sb = vdo.sB;
+  qp.do_sh = vdo.sH;
+  qp.do_sl = vdo.sL;
   if (remap) {
     qp.dq = static_cast<__nv_bfloat16*>(dqh);
     qp.dq_sb = (int64_t)c.Hq * c.L * c.d;
@@ -441,9 +450,9 @@ cp_status_t run_backward(const cp_plan_t* plan, const cp_tensor_t* q, const cp_t
   qp.debug_fault = c.debug_fault;
   const int64_t qgrid = (int64_t)qp.n_chunks * qp.tiles_per_chunk * c.B * c.Hq;
   if (c.d == 128) {
-    CP_TRY(launch_bwd_dq_d<128>(qp, mq, mk, mv, mdo, qgrid, s));
+    CP_TRY(launch_bwd_dq_d<128>(qp, mk, mv, qgrid, s));
   } else {
-    CP_TRY(launch_bwd_dq_d<64>(qp, mq, mk, mv, mdo, qgrid, s));
+    CP_TRY(launch_bwd_dq_d<64>(qp, mk, mv, qgrid, s));
   }
   if (!seq) return CP_OK;
   // all-to-all head -> seq of dK and dV (and of dQ under a two-shard split)
