@@ -21,12 +21,16 @@
 
 using namespace cpattn;
 
-// Streams and events of the host-buffer forward on one device, created at its first call and
-// kept until the plan is destroyed (e_in / e_comp: one pair per block of KV heads).
+// Streams and events of the plan on one device, created at their first use and kept until the
+// plan is destroyed: the host-buffer forward's copy streams (e_in / e_comp: one pair per block
+// of KV heads), and the side stream on which the two-shard ring step runs its second query
+// shard, forked from and joined back into the caller's stream.
 struct HostPipe {
   cudaStream_t s_in = nullptr, s_out = nullptr;
   cudaEvent_t e_start = nullptr, e_done = nullptr;
   std::vector<cudaEvent_t> e_in, e_comp;
+  cudaStream_t s_side = nullptr;
+  cudaEvent_t e_fork = nullptr, e_join = nullptr;
 };
 
 struct cp_plan {
@@ -536,6 +540,9 @@ void cp_attn_plan_destroy(cp_plan_t* plan) {
     if (hp.e_done) cudaEventDestroy(hp.e_done);
     if (hp.s_in) cudaStreamDestroy(hp.s_in);
     if (hp.s_out) cudaStreamDestroy(hp.s_out);
+    if (hp.e_fork) cudaEventDestroy(hp.e_fork);
+    if (hp.e_join) cudaEventDestroy(hp.e_join);
+    if (hp.s_side) cudaStreamDestroy(hp.s_side);
   }
   if (prev >= 0) cudaSetDevice(prev);
   delete plan;
@@ -771,8 +778,20 @@ cp_status_t cp_ring_step(const cp_plan_t* plan, int rank, int step, const cp_ten
     // Two shards per rank (each w = c/2 rows), chunks of a 2N-chunk split: the query rows are
     // rank's shards (a0, a1) in that order, the KV rows rank j's shards (b0, b1).  One launch
     // per query shard covers both KV shards, merged in the kernel; a query shard that sees
-    // neither gets the merge identity.
+    // neither gets the merge identity.  The second shard's launch runs on the plan's side
+    // stream, so the two launches fill each other's last wave; both are ordered after the work
+    // already on the caller's stream, and the caller's stream waits for both.
     const int w = ch / 2;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CP_ERR_CUDA;
+    std::lock_guard<std::mutex> guard(plan->host_mu);  // the side stream's events are reused
+    HostPipe& hp = plan->host_pipes[dev];
+    if (!hp.s_side && cudaStreamCreateWithFlags(&hp.s_side, cudaStreamNonBlocking) != cudaSuccess) return CP_ERR_CUDA;
+    if (!hp.e_fork && cudaEventCreateWithFlags(&hp.e_fork, cudaEventDisableTiming) != cudaSuccess) return CP_ERR_CUDA;
+    if (!hp.e_join && cudaEventCreateWithFlags(&hp.e_join, cudaEventDisableTiming) != cudaSuccess) return CP_ERR_CUDA;
+    if (cudaEventRecord(hp.e_fork, s) != cudaSuccess || cudaStreamWaitEvent(hp.s_side, hp.e_fork, 0) != cudaSuccess)
+      return CP_ERR_CUDA;
+    cp_status_t st = CP_OK;
     auto shards = [&](int r, int& x0, int& x1) {
       x0 = r;
       x1 = c.split == CP_SPLIT_ZIGZAG ? 2 * N - 1 - r : r + N;
@@ -780,18 +799,19 @@ cp_status_t cp_ring_step(const cp_plan_t* plan, int rank, int step, const cp_ten
     int a[2], b[2];
     shards(rank, a[0], a[1]);
     shards(j, b[0], b[1]);
-    for (int hq = 0; hq < 2; ++hq) {
+    for (int hq = 0; hq < 2 && st == CP_OK; ++hq) {
+      const cudaStream_t sh = hq == 0 ? s : hp.s_side;
       int vis[2], nv = 0;
       for (int t = 0; t < 2; ++t)
         if (!c.causal || b[t] <= a[hq]) vis[nv++] = b[t];
       if (nv == 0) {
         const int64_t n = (int64_t)c.B * c.Hq * w * c.d;
-        fill_identity_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+        fill_identity_kernel<<<(unsigned)((n + 255) / 256), 256, 0, sh>>>(
             static_cast<float*>(o_part->data) + (int64_t)hq * w * o_part->stride[2],
             static_cast<float*>(lse_part->data) + (int64_t)hq * w * lse_part->stride[2], c.B, c.Hq, w, c.d,
             o_part->stride[0], o_part->stride[1], o_part->stride[2], lse_part->stride[0], lse_part->stride[1],
             lse_part->stride[2]);
-        if (cudaGetLastError() != cudaSuccess) return CP_ERR_CUDA;
+        if (cudaGetLastError() != cudaSuccess) st = CP_ERR_CUDA;
         continue;
       }
       FwdParams p{};
@@ -803,9 +823,13 @@ cp_status_t cp_ring_step(const cp_plan_t* plan, int rank, int step, const cp_ten
       const int64_t grid = (int64_t)p.pos_per_chunk * p.n_inner;
       FwdOut out{o_part->data, o_part->stride[0], o_part->stride[1], o_part->stride[2], 1,
                  static_cast<float*>(lse_part->data), lse_part->stride[0], lse_part->stride[1], lse_part->stride[2]};
-      CP_TRY(run_fwd_kernel(plan, p, view_of(q), view_of(k), view_of(v), out, grid, s));
+      st = run_fwd_kernel(plan, p, view_of(q), view_of(k), view_of(v), out, grid, sh);
     }
-    return CP_OK;
+    // join: the caller's stream waits for the side stream's launch (also after an error, so
+    // that nothing is left behind on the side stream)
+    if (cudaEventRecord(hp.e_join, hp.s_side) != cudaSuccess || cudaStreamWaitEvent(s, hp.e_join, 0) != cudaSuccess)
+      return CP_ERR_CUDA;
+    return st;
   }
   if (c.causal && j > rank) {
     const int64_t n = (int64_t)c.B * c.Hq * ch * c.d;
