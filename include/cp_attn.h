@@ -209,7 +209,11 @@ cp_status_t cp_layout_head2seq_split(int n_ranks, cp_split_t split, const cp_ten
  * normalised partial P V / l, lse_part [B,Hq,c] fp32 its LSE.  A chunk wholly above the
  * causal diagonal yields O = 0, LSE = -inf (the merge identity).  Under a two-shard split
  * rank r's c rows are its two shards (local order) and the KV rows are rank j's two shards;
- * a query shard that sees neither KV shard gets the identity. */
+ * a query shard that sees neither KV shard gets the identity.  Under a two-shard split the
+ * second query shard's work runs on a stream the plan owns (created at the first such call
+ * on the device, destroyed with the plan), forked from `stream` and joined back into it: work
+ * enqueued on `stream` after the call sees both shards' results.  Calls on one plan enqueue
+ * one at a time (a lock). */
 cp_status_t cp_ring_step(const cp_plan_t* plan, int rank, int step, const cp_tensor_t* q,
                          const cp_tensor_t* k, const cp_tensor_t* v, cp_tensor_t* o_part,
                          cp_tensor_t* lse_part, void* stream);
