@@ -103,7 +103,8 @@ typedef struct {
                            the kernel ends with CP_ERR_TIMEOUT in the status word (nothing
                            faults or hangs): 1 => the forward kernel skips the query-tile load;
                            2 => the backward's dK/dV kernel skips the K/V tile load; 3 => the
-                           backward's dQ kernel skips the Q/dO tile load.  Other values:
+                           backward's dQ kernel never reports its Q/dO rows as stored in TMEM
+                           (its MMA thread's wait for them expires).  Other values:
                            CP_ERR_INVALID_ARG.                                                  */
 } cp_attn_config_t;
 
