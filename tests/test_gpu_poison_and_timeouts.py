@@ -5,8 +5,8 @@ before a call, and the result must equal, bit for bit, the same call on zero-fil
 kernel that read a byte it had not written first -- a workspace word left from nothing, an
 output element assumed zero -- would carry the NaN or the difference into the result.
 
-Bounded waits: a host flag makes one load warp leave out a load, so every wait that depends on
-it expires.  The kernel must then end with CP_ERR_TIMEOUT and the wait site in the plan's status
+Bounded waits: a host flag makes one producer leave out a load (or, in the dQ kernel, the
+report that Q and dO are in TMEM), so every wait that depends on it expires.  The kernel must then end with CP_ERR_TIMEOUT and the wait site in the plan's status
 word, without a fault, and a correct call on the same context must still match the oracle.
 """
 import numpy as np
