@@ -108,3 +108,29 @@ def test_ulysses_forward_and_backward_under_a_split(cuda_lib, split):
         err = np.abs(got - ref)
         assert err.max() <= 2.0 ** -7 * np.abs(ref).max(), f"{split} {name} max-abs {err.max():.3e}"
         assert err.mean() <= 2.0 ** -7 * np.abs(ref).mean(), f"{split} {name} mean-abs {err.mean():.3e}"
+
+
+@pytest.mark.parametrize("split", SPLITS)
+def test_two_shard_step_is_ordered_on_the_callers_stream(cuda_lib, split):
+    """Under a two-shard split the step's second query shard runs on the plan's own stream,
+    forked from the caller's stream and joined back into it.  So work queued on the caller's
+    stream before the call (here: outputs filled with NaN) is seen by both shards, and work
+    queued after it (a copy) sees both shards' final values: bit for bit those of the same
+    step run alone on the default stream."""
+    B, Hq, Hkv, L, d, n = 1, 8, 2, 8192, 128, 4   # shards of 1024 rows, both with work at r = n-1
+    q, k, v = inputs(771, (B, Hq, L, d), (B, Hkv, L, d))
+    plan = Plan(B, Hq, Hkv, L, d, n_cp=n, split=split)
+    tq, tk, tv = to_dev(q), to_dev(k), to_dev(v)
+    r, st = n - 1, 1
+    ref_o, ref_l = plan.ring_step(r, st, tq, tk, tv)
+    torch.cuda.synchronize()
+    ref_o, ref_l = ref_o.clone(), ref_l.clone()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o = torch.full_like(ref_o, float("nan"))
+        lse = torch.full_like(ref_l, float("nan"))
+        plan.ring_step(r, st, tq, tk, tv, o, lse, stream=s)
+        o2, l2 = o.clone(), lse.clone()
+    torch.cuda.synchronize()
+    assert torch.equal(o2, ref_o) and torch.equal(l2, ref_l), f"{split}: the copy after the call saw unfinished rows"
+    assert plan.device_status()[0] == 0
