@@ -177,7 +177,13 @@ __global__ void __launch_bounds__(kMergeThreads) lse_merge_kernel(const MergePar
 
 // ---- backward preprocess: D_i = sum_e dO_ie * O_ie ------------------------------------------
 // 16 lanes per row at d = 128 (8 at d = 64), each loading 16 bytes of dO and of O, then a
-// butterfly shuffle reduction inside the lane group.  Output D [B, H, L] fp32 (head-major).
+// butterfly shuffle reduction inside the lane group.  A lane group takes kDotRows consecutive
+// rows and issues all their loads before any arithmetic (more bytes in flight per thread).
+// Rows are enumerated in the inputs' memory order: heads fastest when o and dout are
+// sequence-major (head stride below position stride), positions fastest otherwise, so
+// neighbouring lane groups read neighbouring memory.  Output D [B, H, L] fp32 (head-major).
+constexpr int kDotRows = 4;
+
 struct DotParams {
   const __nv_bfloat16* o;
   const __nv_bfloat16* dout;
@@ -193,31 +199,63 @@ struct DotParams {
 __global__ void __launch_bounds__(256) rowdot_kernel(const DotParams p) {
   const int lpr = p.d / 8;  // lanes per row (power of two)
   const long long gthread = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long row = gthread / lpr;
+  const long long row0 = (gthread / lpr) * kDotRows;
   const int vec = static_cast<int>(gthread % lpr);
   const long long n_rows = static_cast<long long>(p.B) * p.H * p.L;
-  const bool live = row < n_rows;
-  float acc = 0.f;
-  int b = 0, h = 0, l = 0;
-  if (live) {
-    l = static_cast<int>(row % p.L);
-    h = static_cast<int>((row / p.L) % p.H);
-    b = static_cast<int>(row / (static_cast<long long>(p.L) * p.H));
-    const long long lr = p.split ? split_rank_row(l, p.split, p.n_ranks, p.shard) : l;
-    const uint4 a = reinterpret_cast<const uint4*>(p.o + b * p.o_sb + h * p.o_sh + lr * p.o_sl)[vec];
-    const uint4 g = reinterpret_cast<const uint4*>(p.dout + b * p.g_sb + h * p.g_sh + lr * p.g_sl)[vec];
-    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+  uint4 a[kDotRows], g[kDotRows];
+  int b[kDotRows], h[kDotRows], l[kDotRows];
+  // (fast, slow) index of row0 along the memory order, then carried forward one row at a time
+  const bool seq_major = p.o_sh < p.o_sl;
+  const int n_fast = seq_major ? p.H : p.L, n_slow = seq_major ? p.L : p.H;
+  const long long q1 = row0 / n_fast;
+  int fast = static_cast<int>(row0 - q1 * n_fast);
+  const long long q2 = q1 / n_slow;
+  int slow = static_cast<int>(q1 - q2 * n_slow);
+  int bb = static_cast<int>(q2);
+#pragma unroll
+  for (int u = 0; u < kDotRows; ++u) {
+    const long long row = row0 + u;
+    h[u] = seq_major ? fast : slow;
+    l[u] = seq_major ? slow : fast;
+    b[u] = bb;
+    a[u] = make_uint4(0u, 0u, 0u, 0u);
+    g[u] = a[u];
+    if (row < n_rows) {
+      const long long lr = p.split ? split_rank_row(l[u], p.split, p.n_ranks, p.shard) : l[u];
+      a[u] = reinterpret_cast<const uint4*>(p.o + b[u] * p.o_sb + h[u] * p.o_sh + lr * p.o_sl)[vec];
+      g[u] = reinterpret_cast<const uint4*>(p.dout + b[u] * p.g_sb + h[u] * p.g_sh + lr * p.g_sl)[vec];
+    }
+    if (++fast == n_fast) {
+      fast = 0;
+      if (++slow == n_slow) {
+        slow = 0;
+        ++bb;
+      }
+    }
+  }
+  float acc[kDotRows];
+#pragma unroll
+  for (int u = 0; u < kDotRows; ++u) {
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g[u]);
+    acc[u] = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 x = __bfloat1622float2(a2[e]);
       const float2 y = __bfloat1622float2(g2[e]);
-      acc = fmaf(x.x, y.x, acc);
-      acc = fmaf(x.y, y.y, acc);
+      acc[u] = fmaf(x.x, y.x, acc[u]);
+      acc[u] = fmaf(x.y, y.y, acc[u]);
     }
   }
-  for (int off = lpr >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (live && vec == 0) p.D[b * p.D_sb + h * p.D_sh + l * p.D_sl] = acc;
+  for (int off = lpr >> 1; off > 0; off >>= 1) {
+#pragma unroll
+    for (int u = 0; u < kDotRows; ++u) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], off);
+  }
+  if (vec == 0) {
+#pragma unroll
+    for (int u = 0; u < kDotRows; ++u)
+      if (row0 + u < n_rows) p.D[b[u] * p.D_sb + h[u] * p.D_sh + l[u] * p.D_sl] = acc[u];
+  }
 }
 
 // ---- fill a step-wise partial with the merge identity (O = 0, LSE = -inf) -------------------

@@ -273,8 +273,9 @@ cp_status_t launch_rowdot(const void* o, const int64_t os[3], const void* g, con
   DotParams p{static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(g), D, B, H, L, d,
               os[0], os[1], os[2], gs[0], gs[1], gs[2], (int64_t)H * L, (int64_t)L, 1,
               sp, n_ranks, sp ? L / (2 * n_ranks) : 1};
-  const int64_t threads = (int64_t)B * H * L * (d / 8);
-  if (threads == 0) return CP_OK;
+  const int64_t rows = (int64_t)B * H * L;
+  if (rows == 0) return CP_OK;
+  const int64_t threads = (rows + kDotRows - 1) / kDotRows * (d / 8);
   rowdot_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
